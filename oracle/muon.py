@@ -1,0 +1,129 @@
+"""Muon optimizer step, written out plainly in NumPy (float64, plus float32 where the
+momentum buffer's own precision is the definition).
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by the smoke check and by the
+benchmark's CPU-baseline leg, never by the product path.  It shares no code with
+the CUDA library.
+
+The method, as the autoresearch ``train.py`` review (web3.cnoyu.systems post
+71151920174080, MuonAdamW paragraph) describes it, for one 2-D weight W with
+gradient G and momentum buffer M:
+
+1. Nesterov momentum on the gradient.
+2. Frobenius normalisation of the result (added by the benchmark spec; the page
+   is silent).
+3. Five Newton-Schulz steps with a per-step coefficient triple (a, b, c):
+   tall (rows > cols):  A = X^T X,  X <- a X + X (b A + c A^2)
+   otherwise (wide):    A = X X^T,  X <- a X + (b A + c A^2) X
+4. W <- W - lr * sqrt(max(1, rows/cols)) * O with O the last X (task statement).
+
+Readings taken where the page is silent or open (each is also listed in the
+design notes of the library):
+
+* Nesterov form: the PyTorch-SGD form M <- mu*M + G, U = G + mu*M (new M); with
+  nesterov off, U = M.  The buffer is float32 and each product and sum is rounded
+  on its own (no fused multiply-add), which is what the bit-exact buffer check
+  compares against.
+* Normalisation: X0 = U / (||U||_F + eps), eps added to the norm, not its square.
+* A square matrix takes the wide rule (the page calls "tall" only rows > cols);
+  both rules agree in exact arithmetic.
+* The per-step coefficient table is an input; the page says the values are
+  precomputed ("Polar Express") but prints none.  ``QUINTIC`` repeated five times
+  is the default.
+* No weight decay on this path.
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, Sequence
+
+import numpy as np
+
+# Quintic triple used for every Newton-Schulz step unless a table is passed.
+QUINTIC = (3.4445, -4.7750, 2.0315)
+# Cubic triple of the classical Newton-Schulz polar iteration X <- 1.5X - 0.5 X X^T X;
+# it converges to the polar factor and is used by the pins, not by the method.
+CUBIC = (1.5, -0.5, 0.0)
+
+
+def nesterov_momentum_f32(grad, momentum, mu: float, nesterov: bool = True):
+    """Momentum step on the float32 buffer (autoresearch review, MuonAdamW paragraph:
+    Muon applies Nesterov momentum to the gradient; the buffer has the parameter's
+    shape).
+
+    Returns (M_new float32, U float64).  M_new = fl32(fl32(mu*M) + G): NumPy float32
+    arithmetic rounds the product and the sum separately.  U = G + mu*M_new for
+    Nesterov, else M_new, evaluated in float64 from the float32 values.
+    """
+    g32 = np.asarray(grad, dtype=np.float32)
+    m32 = np.asarray(momentum, dtype=np.float32)
+    mu32 = np.float32(mu)
+    prod = np.multiply(mu32, m32, dtype=np.float32)
+    m_new = np.add(prod, g32, dtype=np.float32)
+    if nesterov:
+        u = g32.astype(np.float64) + np.float64(mu32) * m_new.astype(np.float64)
+    else:
+        u = m_new.astype(np.float64)
+    return m_new, u
+
+
+def frobenius_normalise(u, eps: float):
+    """X0 = U / (||U||_F + eps), float64 (normalisation before the iteration, as the
+    task statement fixes it)."""
+    u = np.asarray(u, dtype=np.float64)
+    norm = math.sqrt(float(np.sum(u * u)))
+    return u / (norm + eps)
+
+
+def newton_schulz(x0, coeffs: Sequence[Sequence[float]]):
+    """Newton-Schulz steps in float64, one per row (a, b, c) of ``coeffs``
+    (autoresearch review, MuonAdamW paragraph: tall rule A = X^T X,
+    X <- aX + X(bA + cA^2); wide rule A = X X^T, X <- aX + (bA + cA^2)X).
+    Rows > cols is tall; everything else takes the wide rule."""
+    x = np.array(x0, dtype=np.float64, copy=True)
+    if x.ndim != 2:
+        raise ValueError("newton_schulz expects a 2-D matrix")
+    tall = x.shape[0] > x.shape[1]
+    for row in coeffs:
+        a, b, c = (float(v) for v in row)
+        if tall:
+            gram = x.T @ x
+            poly = b * gram + c * (gram @ gram)
+            x = a * x + x @ poly
+        else:
+            gram = x @ x.T
+            poly = b * gram + c * (gram @ gram)
+            x = a * x + poly @ x
+    return x
+
+
+def update_scale(rows: int, cols: int) -> float:
+    """sqrt(max(1, rows/cols)), the shape factor of the applied update (task
+    statement; the page gives none)."""
+    return math.sqrt(max(1.0, rows / cols))
+
+
+def muon_step_matrix(w, grad, momentum, *, lr: float, mu: float, nesterov: bool = True,
+                     coeffs: Sequence[Sequence[float]] | None = None, eps: float = 1e-7):
+    """One Muon step for one matrix.
+
+    Returns (W_new float64, M_new float32, O float64).  W_new is the exact
+    W - lr*scale*O; rounding it to the parameter's dtype is the caller's concern.
+    """
+    if coeffs is None:
+        coeffs = [QUINTIC] * 5
+    w64 = np.asarray(w, dtype=np.float64)
+    rows, cols = w64.shape
+    m_new, u = nesterov_momentum_f32(grad, momentum, mu, nesterov)
+    x0 = frobenius_normalise(u, eps)
+    o = newton_schulz(x0, coeffs)
+    w_new = w64 - lr * update_scale(rows, cols) * o
+    return w_new, m_new, o
+
+
+def muon_step(params: Iterable, grads: Iterable, moms: Iterable, **kw):
+    """Muon step over a list of matrices, one after another (no grouping)."""
+    out = []
+    for w, g, m in zip(params, grads, moms):
+        out.append(muon_step_matrix(w, g, m, **kw))
+    return out
