@@ -1,0 +1,148 @@
+/*
+ * muon.h -- C ABI of the B200 (sm_100a) Muon optimizer step.
+ *
+ * The operation (autoresearch train.py review, web3.cnoyu.systems post
+ * 71151920174080, paragraph on the MuonAdamW optimizer): for every 2-D weight W
+ * with gradient G and momentum buffer M,
+ *
+ *   M  <- mu*M + G                      (float32 buffer, product and sum rounded
+ *                                        separately)
+ *   U  <- G + mu*M   (Nesterov)  or  U <- M
+ *   X0 <- U / (||U||_F + eps)
+ *   k = 1..K, tall (rows > cols):  A = X^T X,  X <- a_k X + X (b_k A + c_k A^2)
+ *             otherwise (wide):    A = X X^T,  X <- a_k X + (b_k A + c_k A^2) X
+ *   W  <- W - fl32(lr*sqrt(max(1, rows/cols))) * X_K
+ *
+ * The page fixes the momentum, the five Newton-Schulz steps, the tall/wide rules
+ * and per-step coefficient triples ("Polar Express", values not printed); the
+ * Frobenius normalisation with eps and the update scale come from the method's
+ * task statement.  Newton-Schulz runs on tcgen05 tensor cores (bf16 operands,
+ * fp32 accumulation) in MUON_MODE_BF16 and on fp32 CUDA-core FMAs in
+ * MUON_MODE_FP32_VALIDATE.
+ *
+ * Conventions for every entry point
+ *  - All matrix pointers are DEVICE pointers on the handle's device, row-major and
+ *    contiguous (element (i, j) at i*cols + j), 16-byte aligned.  They stay owned
+ *    by the caller.  No two matrices' pointers may overlap.
+ *  - Work is enqueued on `cuda_stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and the call returns without waiting for it.
+ *  - Argument errors are detected on the host and returned before anything is
+ *    enqueued (MUON_ERR_INVALID_ARG / MUON_ERR_UNSUPPORTED); the detail is
+ *    available from muon_last_error().  A CUDA error while enqueueing returns
+ *    MUON_ERR_CUDA.  A device-side time-out of one of the library's bounded waits
+ *    is reported as MUON_ERR_TIMEOUT by the next call on the handle, or by
+ *    muon_sync / muon_destroy.
+ *  - The library owns a workspace on the device (two bf16 or fp32 copies of every
+ *    matrix, one s x s Gram and one s x s polynomial buffer per matrix with
+ *    s = min(rows, cols), per-matrix norm partials).  It is allocated, with
+ *    cudaMalloc, on the first call with a new list of shapes and mode, and reused
+ *    by later calls with the same list; such calls allocate nothing.  Calls that
+ *    share a handle must not overlap on the GPU (use one stream per handle, or
+ *    one handle per stream).  A handle is not thread-safe.
+ */
+#ifndef MUON_B200_MUON_H
+#define MUON_B200_MUON_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MUON_API __attribute__((visibility("default")))
+#else
+#define MUON_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct muon_handle* muon_handle_t;
+
+typedef enum {
+  MUON_OK = 0,
+  MUON_ERR_INVALID_ARG = 1,  /* null / misaligned / overlapping pointers, bad sizes or values */
+  MUON_ERR_UNSUPPORTED = 2,  /* a combination this build does not implement (e.g. no sm_100 device) */
+  MUON_ERR_OOM = 3,          /* workspace allocation failed */
+  MUON_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed */
+  MUON_ERR_TIMEOUT = 5       /* a bounded device-side wait expired (kernel gave up and returned) */
+} muon_status;
+
+typedef enum { MUON_F32 = 0, MUON_BF16 = 1 } muon_dtype;
+
+typedef enum {
+  MUON_MODE_BF16 = 0,          /* Newton-Schulz on tcgen05 tensor cores, bf16 operands, fp32 accumulate */
+  MUON_MODE_FP32_VALIDATE = 1  /* Newton-Schulz in fp32 storage and fp32 FMA (validation, slow) */
+} muon_mode;
+
+/* One weight matrix.  param: rows*cols of param_dtype, updated in place.  grad:
+ * rows*cols of grad_dtype, read only.  momentum: rows*cols float32, updated in
+ * place.  rows, cols >= 1. */
+typedef struct {
+  void* param;
+  const void* grad;
+  float* momentum;
+  int64_t rows;
+  int64_t cols;
+  muon_dtype param_dtype;
+  muon_dtype grad_dtype;
+} muon_matrix;
+
+/* Creates a handle bound to CUDA device `device`.  Allocates host memory only and
+ * launches no GPU work.  Returns MUON_ERR_INVALID_ARG for a NULL `out` or a device
+ * index out of range, MUON_ERR_UNSUPPORTED if the device is not compute
+ * capability 10.0 (the kernels are built for sm_100a only). */
+MUON_API muon_status muon_init(muon_handle_t* out, int device);
+
+/* One Muon step over `n` matrices (see the operation above).
+ *  lr            learning rate (finite, >= 0)
+ *  momentum      mu in [0, 1)
+ *  nesterov      nonzero: U = G + mu*M_new; zero: U = M_new
+ *  coeffs        HOST pointer to ns_steps rows of (a, b, c) float32, row k used in
+ *                Newton-Schulz step k; NULL = (3.4445, -4.7750, 2.0315) every step
+ *  ns_steps      1..16
+ *  eps           added to the Frobenius norm (finite, >= 0)
+ *  mode          MUON_MODE_BF16 or MUON_MODE_FP32_VALIDATE
+ *  cuda_stream   cudaStream_t the work is enqueued on
+ * Every matrix is processed independently; their order does not matter.  The
+ * applied factor per matrix is the float32 rounding of lr*sqrt(max(1,rows/cols))
+ * computed in double, and the new weight is fl32(W - fl32(factor*O)) rounded to
+ * nearest-even into param_dtype. */
+MUON_API muon_status muon_step(muon_handle_t h, const muon_matrix* mats, int n,
+                      float lr, float momentum, int nesterov,
+                      const float* coeffs, int ns_steps, float eps,
+                      muon_mode mode, void* cuda_stream);
+
+/* Newton-Schulz part alone: o_out[i] = X_K of X0 = x_in[i] / (||x_in[i]||_F + eps)
+ * for n matrices of shape rows[i] x cols[i].  x_in and o_out are DEVICE pointers
+ * of `dtype`; o_out must not overlap any input.  rows, cols, x_in and o_out are
+ * HOST arrays of length n.  Other arguments as in muon_step. */
+MUON_API muon_status muon_newton_schulz(muon_handle_t h, const void* const* x_in, void* const* o_out,
+                               const int64_t* rows, const int64_t* cols, int n,
+                               muon_dtype dtype, const float* coeffs, int ns_steps,
+                               float eps, muon_mode mode, void* cuda_stream);
+
+/* Waits for the handle's last enqueued work and returns its device-side status
+ * (MUON_OK or MUON_ERR_TIMEOUT), clearing it. */
+MUON_API muon_status muon_sync(muon_handle_t h);
+
+/* Bytes of device workspace the handle currently holds. */
+MUON_API int64_t muon_workspace_bytes(muon_handle_t h);
+
+/* Number of kernel launches the last muon_step / muon_newton_schulz enqueued. */
+MUON_API int muon_last_launch_count(muon_handle_t h);
+
+/* Waits for outstanding work, frees the workspace and the handle.  Returns the
+ * pending device-side status.  NULL is accepted and returns MUON_OK. */
+MUON_API muon_status muon_destroy(muon_handle_t h);
+
+/* Static description of a status code. */
+MUON_API const char* muon_status_string(muon_status s);
+
+/* Detail of the last error on this handle (empty string if none).  The pointer
+ * stays valid until the next call on the handle. */
+MUON_API const char* muon_last_error(muon_handle_t h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUON_B200_MUON_H */

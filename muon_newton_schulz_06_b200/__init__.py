@@ -1,0 +1,231 @@
+"""Python binding of the Muon C ABI (``include/muon.h``): argument marshalling only.
+
+Every step of the optimizer runs in ``libmuon_b200.so`` (sm_100a kernels).  There is
+no fallback: if the library is missing or the device is not a B200-class GPU, the
+calls raise.
+
+    h = muon_init(0)
+    muon_step(h, params, grads, moms, lr=0.02, momentum=0.95)   # lists of CUDA tensors
+    muon_destroy(h)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmuon_b200.so")
+
+MUON_OK = 0
+MUON_ERR_INVALID_ARG = 1
+MUON_ERR_UNSUPPORTED = 2
+MUON_ERR_OOM = 3
+MUON_ERR_CUDA = 4
+MUON_ERR_TIMEOUT = 5
+
+MUON_F32 = 0
+MUON_BF16 = 1
+MUON_MODE_BF16 = 0
+MUON_MODE_FP32_VALIDATE = 1
+
+EXPORTED = ("muon_init", "muon_step", "muon_newton_schulz", "muon_sync", "muon_workspace_bytes",
+            "muon_last_launch_count", "muon_destroy", "muon_status_string", "muon_last_error")
+
+
+class MuonError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(msg)
+        self.code = code
+
+
+class muon_matrix(ctypes.Structure):
+    _fields_ = [("param", ctypes.c_void_p), ("grad", ctypes.c_void_p), ("momentum", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("param_dtype", ctypes.c_int), ("grad_dtype", ctypes.c_int)]
+
+
+_lib_handle = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Loads libmuon_b200.so (raises if it has not been built)."""
+    global _lib_handle
+    if _lib_handle is not None:
+        return _lib_handle
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m muon_newton_schulz_06_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+    lib.muon_init.argtypes = [ctypes.POINTER(vp), i32]
+    lib.muon_init.restype = i32
+    lib.muon_step.argtypes = [vp, ctypes.POINTER(muon_matrix), i32, f32, f32, i32, ctypes.POINTER(f32), i32,
+                              f32, i32, vp]
+    lib.muon_step.restype = i32
+    lib.muon_newton_schulz.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(i64),
+                                       ctypes.POINTER(i64), i32, i32, ctypes.POINTER(f32), i32, f32, i32, vp]
+    lib.muon_newton_schulz.restype = i32
+    lib.muon_sync.argtypes = [vp]
+    lib.muon_sync.restype = i32
+    lib.muon_workspace_bytes.argtypes = [vp]
+    lib.muon_workspace_bytes.restype = i64
+    lib.muon_last_launch_count.argtypes = [vp]
+    lib.muon_last_launch_count.restype = i32
+    lib.muon_destroy.argtypes = [vp]
+    lib.muon_destroy.restype = i32
+    lib.muon_status_string.argtypes = [i32]
+    lib.muon_status_string.restype = ctypes.c_char_p
+    lib.muon_last_error.argtypes = [vp]
+    lib.muon_last_error.restype = ctypes.c_char_p
+    _lib_handle = lib
+    return lib
+
+
+def muon_status_string(code: int) -> str:
+    return load_library().muon_status_string(int(code)).decode()
+
+
+def _check(code: int, handle=None):
+    if code != MUON_OK:
+        lib = load_library()
+        detail = lib.muon_last_error(handle).decode() if handle is not None else ""
+        raise MuonError(code, f"{muon_status_string(code)}" + (f" ({detail})" if detail else ""))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MUON_BF16
+    if t.dtype == torch.float32:
+        return MUON_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _check_tensor(t: torch.Tensor, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dim() != 2 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous 2-D tensor")
+
+
+def _coeff_array(coeffs, ns_steps):
+    if coeffs is None:
+        return None
+    flat = [float(v) for row in coeffs for v in row]
+    if len(flat) != 3 * ns_steps:
+        raise ValueError("coeffs must hold ns_steps rows of (a, b, c)")
+    return (ctypes.c_float * len(flat))(*flat)
+
+
+def _mode_code(mode) -> int:
+    if mode in ("bf16", MUON_MODE_BF16):
+        return MUON_MODE_BF16
+    if mode in ("fp32", "fp32_validate", MUON_MODE_FP32_VALIDATE):
+        return MUON_MODE_FP32_VALIDATE
+    raise ValueError(f"unknown mode {mode!r}")
+
+
+def _stream_ptr(stream, device) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def muon_init(device: int = 0):
+    """Returns an opaque handle bound to CUDA device ``device``."""
+    h = ctypes.c_void_p()
+    _check(load_library().muon_init(ctypes.byref(h), int(device)))
+    return h
+
+
+def muon_step(handle, params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
+              moms: Sequence[torch.Tensor], lr: float, momentum: float = 0.95, nesterov: bool = True,
+              coeffs=None, ns_steps: int = 5, eps: float = 1e-7, mode="bf16", stream=None) -> None:
+    """One Muon step over matched lists of parameters (bf16/fp32, updated in place),
+    gradients (bf16/fp32) and float32 momentum buffers (updated in place)."""
+    n = len(params)
+    if len(grads) != n or len(moms) != n:
+        raise ValueError("params, grads and moms must have the same length")
+    arr = (muon_matrix * max(n, 1))()
+    for i, (w, g, m) in enumerate(zip(params, grads, moms)):
+        _check_tensor(w, "param")
+        _check_tensor(g, "grad")
+        _check_tensor(m, "momentum")
+        if m.dtype != torch.float32:
+            raise TypeError("momentum buffers must be float32")
+        if g.shape != w.shape or m.shape != w.shape:
+            raise ValueError(f"matrix {i}: param, grad and momentum shapes differ")
+        arr[i] = muon_matrix(w.data_ptr(), g.data_ptr(), m.data_ptr(), w.shape[0], w.shape[1],
+                             _dtype_code(w), _dtype_code(g))
+    dev = params[0].device if n else torch.device("cuda")
+    c = _coeff_array(coeffs, ns_steps)
+    _check(load_library().muon_step(handle, arr, n, float(lr), float(momentum), 1 if nesterov else 0, c,
+                                    int(ns_steps), float(eps), _mode_code(mode), _stream_ptr(stream, dev)),
+           handle)
+
+
+def muon_newton_schulz(handle, xs: Sequence[torch.Tensor], outs: Sequence[torch.Tensor], coeffs=None,
+                       ns_steps: int = 5, eps: float = 1e-7, mode="bf16", stream=None) -> None:
+    """outs[i] <- Newton-Schulz of xs[i] / (||xs[i]||_F + eps); xs and outs share a dtype."""
+    n = len(xs)
+    if len(outs) != n:
+        raise ValueError("xs and outs must have the same length")
+    if n == 0:
+        return
+    dt = _dtype_code(xs[0])
+    xin = (ctypes.c_void_p * n)()
+    xout = (ctypes.c_void_p * n)()
+    rows = (ctypes.c_int64 * n)()
+    cols = (ctypes.c_int64 * n)()
+    for i, (x, o) in enumerate(zip(xs, outs)):
+        _check_tensor(x, "x")
+        _check_tensor(o, "out")
+        if _dtype_code(x) != dt or _dtype_code(o) != dt:
+            raise TypeError("all inputs and outputs must share one dtype")
+        if o.shape != x.shape:
+            raise ValueError(f"matrix {i}: output shape differs from input shape")
+        xin[i], xout[i], rows[i], cols[i] = x.data_ptr(), o.data_ptr(), x.shape[0], x.shape[1]
+    c = _coeff_array(coeffs, ns_steps)
+    _check(load_library().muon_newton_schulz(handle, xin, xout, rows, cols, n, dt, c, int(ns_steps), float(eps),
+                                             _mode_code(mode), _stream_ptr(stream, xs[0].device)), handle)
+
+
+def muon_sync(handle) -> None:
+    _check(load_library().muon_sync(handle), handle)
+
+
+def muon_workspace_bytes(handle) -> int:
+    return int(load_library().muon_workspace_bytes(handle))
+
+
+def muon_last_launch_count(handle) -> int:
+    return int(load_library().muon_last_launch_count(handle))
+
+
+def muon_destroy(handle) -> None:
+    _check(load_library().muon_destroy(handle))
+
+
+class Muon:
+    """Small convenience wrapper owning one handle."""
+
+    def __init__(self, device: int = 0):
+        self.handle = muon_init(device)
+
+    def step(self, params, grads, moms, **kw):
+        muon_step(self.handle, params, grads, moms, **kw)
+
+    def newton_schulz(self, xs, outs, **kw):
+        muon_newton_schulz(self.handle, xs, outs, **kw)
+
+    def close(self):
+        if self.handle is not None:
+            muon_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

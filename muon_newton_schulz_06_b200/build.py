@@ -1,0 +1,47 @@
+"""Builds the sm_100a shared library libmuon_b200.so next to this file.
+
+    python -m muon_newton_schulz_06_b200.build [--verbose-ptxas]
+
+nvcc compiles every kernel for sm_100a only (tcgen05 / TMA / TMEM instructions) and
+links the CUDA runtime statically, so the library needs no libcudart at load time.
+"""
+import glob
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+LIB = os.path.join(HERE, "libmuon_b200.so")
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def sources():
+    return sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
+
+
+def up_to_date():
+    if not os.path.exists(LIB):
+        return False
+    t = os.path.getmtime(LIB)
+    deps = sources() + glob.glob(os.path.join(HERE, "csrc", "*.h")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
+    return all(os.path.getmtime(d) <= t for d in deps)
+
+
+def build(verbose_ptxas=False, force=False):
+    if not force and up_to_date():
+        return LIB
+    nvcc = os.environ.get("NVCC", "nvcc")
+    cmd = [nvcc, *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
+           "-Xcompiler", "-fvisibility=hidden", "-cudart", "static",
+           "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp", *sources()]
+    if verbose_ptxas:
+        cmd[1:1] = ["-Xptxas", "-v"]
+    subprocess.run(cmd, check=True)
+    os.replace(LIB + ".tmp", LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    build(verbose_ptxas="--verbose-ptxas" in sys.argv, force=True)
+    print(LIB)

@@ -1,0 +1,679 @@
+// Host side of the Muon C ABI: argument checks, the plan (shape groups, workspace
+// layout, tile lists, TMA tensor maps) and the stream-ordered launch sequence
+//
+//   momentum_norm -> { Gram -> Poly -> Update } x ns_steps -> apply
+//
+// (17 launches for five steps when the shapes fit one launch per phase).  Matrices
+// of equal wide-orientation shape (s, L) = (min(r,c), max(r,c)) are stacked into one
+// group, the device analogue of the per-shape-group stacking of the momentum
+// buffers that the autoresearch train.py review describes for MuonAdamW.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/muon.h"
+#include "muon_internal.h"
+
+using namespace muon;
+
+namespace {
+
+constexpr float kDefaultCoeffs[3] = {3.4445f, -4.7750f, 2.0315f};
+constexpr int64_t kMaxDim = int64_t(1) << 24;
+constexpr int kMaxNsSteps = 16;
+constexpr int kMaxMatrices = 65535;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+int round8(int v) { return (v + 7) / 8 * 8; }
+
+struct GroupPlan {
+  int s = 0, L = 0, n = 0;
+  int ld_x = 0, ld_s = 0;
+  int gid_base = 0;
+  size_t off_x[2] = {0, 0};
+  size_t off_gram = 0, off_poly = 0;
+};
+
+struct MatPlan {
+  int group = 0, idx = 0;
+  int64_t rows = 0, cols = 0;
+  bool transposed = false;
+  int n_units = 0, part_base = 0, tiles_c = 0;
+};
+
+struct ChunkPlan {
+  int g_begin = 0, g_end = 0;
+  size_t off_tiles[3] = {0, 0, 0};
+  int n_tiles[3] = {0, 0, 0};
+};
+
+struct Plan {
+  bool valid = false;
+  muon_mode mode = MUON_MODE_BF16;
+  std::vector<int64_t> sig;  // rows, cols pairs
+  std::vector<GroupPlan> groups;
+  std::vector<MatPlan> mats;
+  std::vector<ChunkPlan> chunks;
+  std::vector<TcTile> tiles;  // host copy of every chunk's tile lists
+  size_t off_partials = 0, off_counters = 0, off_scale = 0, off_tiles = 0, bytes = 0;
+  int total_units = 0;
+  // TMA maps per group (bf16 mode): X K-major (ping/pong), X MN-major (ping/pong), Gram, Poly
+  std::vector<CUtensorMap> map_xk[2], map_xmn[2], map_gram, map_poly;
+};
+
+}  // namespace
+
+struct muon_handle {
+  int device = 0;
+  int sm_count = 148;
+  std::string err;
+  int last_launches = 0;
+  EncodeTiledFn encode = nullptr;
+  char* ws = nullptr;
+  size_t ws_bytes = 0;
+  int* dev_status = nullptr;
+  int* host_status = nullptr;
+  cudaEvent_t status_event = nullptr;
+  bool status_pending = false;
+  Plan plan;
+};
+
+namespace {
+
+muon_status fail(muon_handle* h, muon_status st, const char* fmt, ...) {
+  if (h) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    h->err = buf;
+  }
+  return st;
+}
+
+muon_status cuda_fail(muon_handle* h, cudaError_t e, const char* what) {
+  return fail(h, MUON_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Restores the caller's current device on scope exit.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    ok = cudaSetDevice(dev) == cudaSuccess;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+bool finite(float v) { return std::isfinite(v); }
+
+struct Range {
+  uintptr_t lo, hi;
+  int mat;
+};
+
+muon_status check_overlaps(muon_handle* h, std::vector<Range>& rs) {
+  std::sort(rs.begin(), rs.end(), [](const Range& a, const Range& b) { return a.lo < b.lo; });
+  for (size_t i = 1; i < rs.size(); ++i)
+    if (rs[i].lo < rs[i - 1].hi)
+      return fail(h, MUON_ERR_INVALID_ARG, "buffers of matrices %d and %d overlap", rs[i - 1].mat, rs[i].mat);
+  return MUON_OK;
+}
+
+muon_status check_coeffs(muon_handle* h, const float* coeffs, int ns_steps) {
+  if (ns_steps < 1 || ns_steps > kMaxNsSteps)
+    return fail(h, MUON_ERR_INVALID_ARG, "ns_steps %d outside 1..%d", ns_steps, kMaxNsSteps);
+  if (coeffs)
+    for (int i = 0; i < 3 * ns_steps; ++i)
+      if (!finite(coeffs[i])) return fail(h, MUON_ERR_INVALID_ARG, "coefficient %d is not finite", i);
+  return MUON_OK;
+}
+
+// ------------------------------------------------------------------ plan
+
+void sort_tiles(std::vector<TcTile>& t, const std::vector<GroupPlan>& groups, int phase) {
+  auto cost = [&](const TcTile& x) {
+    const GroupPlan& g = groups[x.group];
+    return (int64_t)(phase == kPhaseGram ? g.L : g.s);
+  };
+  std::stable_sort(t.begin(), t.end(), [&](const TcTile& a, const TcTile& b) { return cost(a) > cost(b); });
+}
+
+muon_status encode_map(muon_handle* h, CUtensorMap* map, void* base, int inner, int rows, int n, int ld,
+                       int box_inner, int box_rows) {
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)n};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)ld * 2 * (cuuint64_t)rows};
+  cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = h->encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(h, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MUON_OK;
+}
+
+muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols, int n, muon_mode mode,
+                       cudaStream_t st) {
+  Plan& P = h->plan;
+  P = Plan();
+  P.mode = mode;
+  const size_t esz = (mode == MUON_MODE_BF16) ? 2 : 4;
+  P.sig.resize(2 * (size_t)n);
+  P.mats.resize(n);
+  for (int i = 0; i < n; ++i) {
+    P.sig[2 * i] = rows[i];
+    P.sig[2 * i + 1] = cols[i];
+    const int s = (int)std::min(rows[i], cols[i]);
+    const int L = (int)std::max(rows[i], cols[i]);
+    int gi = -1;
+    for (size_t g = 0; g < P.groups.size(); ++g)
+      if (P.groups[g].s == s && P.groups[g].L == L) gi = (int)g;
+    if (gi < 0) {
+      GroupPlan g;
+      g.s = s;
+      g.L = L;
+      g.ld_x = round8(L);
+      g.ld_s = round8(s);
+      P.groups.push_back(g);
+      gi = (int)P.groups.size() - 1;
+    }
+    MatPlan& m = P.mats[i];
+    m.group = gi;
+    m.idx = P.groups[gi].n++;
+    m.rows = rows[i];
+    m.cols = cols[i];
+    m.transposed = rows[i] > cols[i];
+    m.tiles_c = (int)((cols[i] + kEwTile - 1) / kEwTile);
+    m.n_units = (int)((rows[i] + kEwTile - 1) / kEwTile) * m.tiles_c;
+    m.part_base = P.total_units;
+    P.total_units += m.n_units;
+  }
+  // global matrix index = group-major order
+  int gid = 0;
+  for (auto& g : P.groups) {
+    g.gid_base = gid;
+    gid += g.n;
+  }
+  // workspace layout
+  size_t off = 0;
+  for (auto& g : P.groups) {
+    const size_t xbytes = (size_t)g.n * g.s * g.ld_x * esz;
+    const size_t sbytes = (size_t)g.n * g.s * g.ld_s * esz;
+    g.off_x[0] = off; off = align_up(off + xbytes, 1024);
+    g.off_x[1] = off; off = align_up(off + xbytes, 1024);
+    g.off_gram = off; off = align_up(off + sbytes, 1024);
+    g.off_poly = off; off = align_up(off + sbytes, 1024);
+  }
+  P.off_partials = off; off = align_up(off + (size_t)P.total_units * 4, 256);
+  P.off_counters = off; off = align_up(off + (size_t)n * 4, 256);
+  P.off_scale = off; off = align_up(off + (size_t)n * 4, 256);
+  // tile lists (tensor-core path)
+  if (mode == MUON_MODE_BF16) {
+    for (int g0 = 0; g0 < (int)P.groups.size(); g0 += kMaxGroups) {
+      ChunkPlan c;
+      c.g_begin = g0;
+      c.g_end = std::min((int)P.groups.size(), g0 + kMaxGroups);
+      std::vector<TcTile> syrk, upd;
+      for (int gg = c.g_begin; gg < c.g_end; ++gg) {
+        const GroupPlan& g = P.groups[gg];
+        const int mb = (g.s + kBM - 1) / kBM, nb_s = (g.s + kBN - 1) / kBN, nb_l = (g.L + kBN - 1) / kBN;
+        for (int m = 0; m < g.n; ++m) {
+          for (int bi = 0; bi < mb; ++bi)
+            for (int bj = 0; bj < nb_s; ++bj)
+              if (bj * kBN + kBN - 1 >= bi * kBM)  // touches the upper triangle
+                syrk.push_back(TcTile{(uint16_t)(gg - c.g_begin), (uint16_t)m, (uint16_t)bi, (uint16_t)bj});
+          for (int bi = 0; bi < mb; ++bi)
+            for (int bj = 0; bj < nb_l; ++bj)
+              upd.push_back(TcTile{(uint16_t)(gg - c.g_begin), (uint16_t)m, (uint16_t)bi, (uint16_t)bj});
+        }
+      }
+      std::vector<GroupPlan> cg(P.groups.begin() + c.g_begin, P.groups.begin() + c.g_end);
+      std::vector<TcTile> lists[3] = {syrk, syrk, upd};
+      for (int ph = 0; ph < 3; ++ph) {
+        sort_tiles(lists[ph], cg, ph);
+        c.off_tiles[ph] = P.tiles.size();
+        c.n_tiles[ph] = (int)lists[ph].size();
+        P.tiles.insert(P.tiles.end(), lists[ph].begin(), lists[ph].end());
+      }
+      P.chunks.push_back(c);
+    }
+  }
+  P.off_tiles = off;
+  off = align_up(off + P.tiles.size() * sizeof(TcTile), 256);
+  P.bytes = off;
+
+  // (re)allocate the workspace
+  if (P.bytes > h->ws_bytes) {
+    if (h->ws) {
+      cudaError_t e = cudaStreamSynchronize(st);
+      if (e != cudaSuccess) return cuda_fail(h, e, "synchronize before workspace reallocation");
+      cudaFree(h->ws);
+      h->ws = nullptr;
+      h->ws_bytes = 0;
+    }
+    void* p = nullptr;
+    if (cudaMalloc(&p, P.bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(h, MUON_ERR_OOM, "workspace allocation of %zu bytes failed", P.bytes);
+    }
+    h->ws = static_cast<char*>(p);
+    h->ws_bytes = P.bytes;
+  }
+  cudaError_t e = cudaMemsetAsync(h->ws + P.off_counters, 0, (size_t)n * 4, st);
+  if (e != cudaSuccess) return cuda_fail(h, e, "counter reset");
+  if (!P.tiles.empty()) {
+    e = cudaMemcpyAsync(h->ws + P.off_tiles, P.tiles.data(), P.tiles.size() * sizeof(TcTile),
+                        cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "tile list upload");
+    e = cudaStreamSynchronize(st);  // the host vector must outlive the copy
+    if (e != cudaSuccess) return cuda_fail(h, e, "tile list upload");
+  }
+  if (mode == MUON_MODE_BF16) {
+    const size_t ng = P.groups.size();
+    for (int b = 0; b < 2; ++b) {
+      P.map_xk[b].resize(ng);
+      P.map_xmn[b].resize(ng);
+    }
+    P.map_gram.resize(ng);
+    P.map_poly.resize(ng);
+    for (size_t gg = 0; gg < ng; ++gg) {
+      const GroupPlan& g = P.groups[gg];
+      muon_status s;
+      for (int b = 0; b < 2; ++b) {
+        if ((s = encode_map(h, &P.map_xk[b][gg], h->ws + g.off_x[b], g.L, g.s, g.n, g.ld_x, kBK, kBM))) return s;
+        if ((s = encode_map(h, &P.map_xmn[b][gg], h->ws + g.off_x[b], g.L, g.s, g.n, g.ld_x, 64, kBK))) return s;
+      }
+      if ((s = encode_map(h, &P.map_gram[gg], h->ws + g.off_gram, g.s, g.s, g.n, g.ld_s, kBK, kBM))) return s;
+      if ((s = encode_map(h, &P.map_poly[gg], h->ws + g.off_poly, g.s, g.s, g.n, g.ld_s, kBK, kBM))) return s;
+    }
+  }
+  P.valid = true;
+  return MUON_OK;
+}
+
+bool plan_matches(const Plan& P, const int64_t* rows, const int64_t* cols, int n, muon_mode mode) {
+  if (!P.valid || P.mode != mode || P.sig.size() != 2 * (size_t)n) return false;
+  for (int i = 0; i < n; ++i)
+    if (P.sig[2 * i] != rows[i] || P.sig[2 * i + 1] != cols[i]) return false;
+  return true;
+}
+
+// ------------------------------------------------------------------ launches
+
+struct CallMat {
+  void* param;        // param (step) / x_in (Newton-Schulz entry)
+  const void* grad;
+  float* mom;
+  void* out;          // o_out (Newton-Schulz entry)
+  bool param_bf16, grad_bf16;
+  float lrs;
+};
+
+void* work_ptr(muon_handle* h, const MatPlan& m, int buf) {
+  const Plan& P = h->plan;
+  const GroupPlan& g = P.groups[m.group];
+  const size_t esz = (P.mode == MUON_MODE_BF16) ? 2 : 4;
+  return h->ws + g.off_x[buf] + (size_t)m.idx * g.s * g.ld_x * esz;
+}
+
+muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, bool momentum_pass,
+                               int out_kind, int work_buf, float mu, int nesterov, float eps, cudaStream_t st) {
+  const Plan& P = h->plan;
+  const int n = (int)cm.size();
+  const bool f32 = (P.mode == MUON_MODE_FP32_VALIDATE);
+  for (int b = 0; b < n; b += kMaxMatsPerLaunch) {
+    EwParams* ep = new EwParams();
+    std::memset(ep, 0, sizeof(EwParams));
+    ep->n_mats = std::min(kMaxMatsPerLaunch, n - b);
+    ep->mu = mu;
+    ep->nesterov = nesterov;
+    ep->use_momentum = (momentum_pass && cm[b].mom != nullptr) ? 1 : 0;
+    ep->eps = eps;
+    ep->partials = reinterpret_cast<float*>(h->ws + P.off_partials);
+    ep->counters = reinterpret_cast<unsigned*>(h->ws + P.off_counters);
+    ep->scale = reinterpret_cast<float*>(h->ws + P.off_scale);
+    int units = 0;
+    for (int j = 0; j < ep->n_mats; ++j) {
+      const int i = b + j;
+      const MatPlan& m = P.mats[i];
+      const GroupPlan& g = P.groups[m.group];
+      EwMat& e = ep->mats[j];
+      const bool export_pass = !momentum_pass && out_kind == kEwExport;
+      e.param = export_pass ? cm[i].out : cm[i].param;
+      e.grad = cm[i].grad;
+      e.mom = cm[i].mom;
+      e.work = work_ptr(h, m, work_buf);
+      e.rows = (int32_t)m.rows;
+      e.cols = (int32_t)m.cols;
+      e.ld = g.ld_x;
+      e.tiles_c = m.tiles_c;
+      e.unit_begin = units;
+      e.gid = g.gid_base + m.idx;
+      e.part_base = m.part_base;
+      e.n_units = m.n_units;
+      e.transposed = m.transposed ? 1 : 0;
+      e.vec_ok = (m.cols % 8 == 0) ? 1 : 0;
+      e.param_bf16 = cm[i].param_bf16 ? 1 : 0;
+      e.grad_bf16 = cm[i].grad_bf16 ? 1 : 0;
+      e.lrs = cm[i].lrs;
+      units += m.n_units;
+    }
+    ep->total_units = units;
+    const int grid = std::max(1, std::min(units, h->sm_count * 8));
+    cudaError_t err = momentum_pass ? launch_momentum_norm(*ep, f32, grid, st)
+                                    : launch_apply(*ep, f32, out_kind, grid, st);
+    delete ep;
+    if (err != cudaSuccess) return cuda_fail(h, err, momentum_pass ? "momentum/norm launch" : "apply launch");
+    h->last_launches++;
+  }
+  return MUON_OK;
+}
+
+muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, cudaStream_t st) {
+  const Plan& P = h->plan;
+  float* scale = reinterpret_cast<float*>(h->ws + P.off_scale);
+  if (P.mode == MUON_MODE_FP32_VALIDATE) {
+    for (int k = 0; k < ns_steps; ++k) {
+      const int cur = k & 1;
+      const float* c = coeffs ? coeffs + 3 * k : kDefaultCoeffs;
+      for (size_t i = 0; i < P.mats.size(); ++i) {
+        const MatPlan& m = P.mats[i];
+        const GroupPlan& g = P.groups[m.group];
+        F32Mat f;
+        f.x_cur = reinterpret_cast<float*>(work_ptr(h, m, cur));
+        f.x_next = reinterpret_cast<float*>(work_ptr(h, m, cur ^ 1));
+        f.gram = reinterpret_cast<float*>(h->ws + g.off_gram + (size_t)m.idx * g.s * g.ld_s * 4);
+        f.poly = reinterpret_cast<float*>(h->ws + g.off_poly + (size_t)m.idx * g.s * g.ld_s * 4);
+        f.s = g.s; f.L = g.L; f.ld_x = g.ld_x; f.ld_s = g.ld_s; f.gid = g.gid_base + m.idx;
+        cudaError_t e = launch_f32_gram(f, k == 0, scale, st);
+        if (e == cudaSuccess) e = launch_f32_poly(f, c[1], c[2], st);
+        if (e == cudaSuccess) e = launch_f32_update(f, k == 0, scale, c[0], st);
+        if (e != cudaSuccess) return cuda_fail(h, e, "fp32 Newton-Schulz launch");
+        h->last_launches += 3;
+      }
+    }
+    return MUON_OK;
+  }
+  TcParams* tp = new TcParams();
+  for (int k = 0; k < ns_steps; ++k) {
+    const int cur = k & 1;
+    const float* c = coeffs ? coeffs + 3 * k : kDefaultCoeffs;
+    for (int ph = 0; ph < 3; ++ph) {
+      for (const ChunkPlan& ch : P.chunks) {
+        std::memset(tp, 0, sizeof(TcParams));
+        for (int gg = ch.g_begin; gg < ch.g_end; ++gg) {
+          const int li = gg - ch.g_begin;
+          const GroupPlan& g = P.groups[gg];
+          TcGroup& t = tp->g[li];
+          t.s = g.s; t.L = g.L; t.ld_x = g.ld_x; t.ld_s = g.ld_s; t.gid_base = g.gid_base;
+          t.x_cur = reinterpret_cast<__nv_bfloat16*>(h->ws + g.off_x[cur]);
+          t.x_next = reinterpret_cast<__nv_bfloat16*>(h->ws + g.off_x[cur ^ 1]);
+          t.gram = reinterpret_cast<__nv_bfloat16*>(h->ws + g.off_gram);
+          t.poly = reinterpret_cast<__nv_bfloat16*>(h->ws + g.off_poly);
+          if (ph == kPhaseGram) {
+            tp->map_a[li] = P.map_xk[cur][gg];
+          } else if (ph == kPhasePoly) {
+            tp->map_a[li] = P.map_gram[gg];
+          } else {
+            tp->map_a[li] = P.map_poly[gg];
+            tp->map_b[li] = P.map_xmn[cur][gg];
+          }
+        }
+        tp->tiles = reinterpret_cast<const TcTile*>(h->ws + P.off_tiles) + ch.off_tiles[ph];
+        tp->n_tiles = ch.n_tiles[ph];
+        tp->first_iter = (k == 0) ? 1 : 0;
+        tp->ca = c[0];
+        tp->cb = c[1];
+        tp->cc = c[2];
+        tp->scale = scale;
+        tp->status = h->dev_status;
+        const int grid = std::max(1, std::min(tp->n_tiles, h->sm_count));
+        cudaError_t e = launch_tc(ph, *tp, grid, st);
+        if (e != cudaSuccess) {
+          delete tp;
+          return cuda_fail(h, e, "tensor-core Newton-Schulz launch");
+        }
+        h->last_launches++;
+      }
+    }
+  }
+  delete tp;
+  return MUON_OK;
+}
+
+muon_status ensure_status(muon_handle* h) {
+  if (h->dev_status) return MUON_OK;
+  cudaError_t e = cudaMalloc(&h->dev_status, sizeof(int));
+  if (e != cudaSuccess) return fail(h, MUON_ERR_OOM, "status word allocation failed");
+  e = cudaMemset(h->dev_status, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaHostAlloc(&h->host_status, sizeof(int), cudaHostAllocDefault);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->status_event, cudaEventDisableTiming);
+  if (e != cudaSuccess) return cuda_fail(h, e, "status set-up");
+  *h->host_status = 0;
+  return MUON_OK;
+}
+
+// Reports a device-side time-out of earlier work, if its status copy has landed.
+muon_status poll_status(muon_handle* h, bool wait) {
+  if (!h->status_pending) return MUON_OK;
+  cudaError_t e = wait ? cudaEventSynchronize(h->status_event) : cudaEventQuery(h->status_event);
+  if (e == cudaErrorNotReady) {
+    cudaGetLastError();
+    return MUON_OK;
+  }
+  if (e != cudaSuccess) return cuda_fail(h, e, "status event");
+  h->status_pending = false;
+  if (*h->host_status != kDevOk) {
+    *h->host_status = kDevOk;
+    cudaMemset(h->dev_status, 0, sizeof(int));
+    return fail(h, MUON_ERR_TIMEOUT, "a device-side wait of an earlier call timed out");
+  }
+  return MUON_OK;
+}
+
+muon_status finish_call(muon_handle* h, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(st, &cs);
+  if (cs != cudaStreamCaptureStatusNone) return MUON_OK;
+  cudaError_t e = cudaMemcpyAsync(h->host_status, h->dev_status, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaEventRecord(h->status_event, st);
+  if (e != cudaSuccess) return cuda_fail(h, e, "status copy");
+  h->status_pending = true;
+  return MUON_OK;
+}
+
+muon_status run(muon_handle* h, const std::vector<CallMat>& cm, const int64_t* rows, const int64_t* cols,
+                bool step, float mu, int nesterov, const float* coeffs, int ns_steps, float eps,
+                muon_mode mode, cudaStream_t st) {
+  const int n = (int)cm.size();
+  DeviceGuard dg(h->device);
+  if (!dg.ok) return fail(h, MUON_ERR_CUDA, "cannot select device %d", h->device);
+  muon_status s = ensure_status(h);
+  if (s) return s;
+  s = poll_status(h, false);
+  if (s) return s;
+  h->last_launches = 0;
+  if (!plan_matches(h->plan, rows, cols, n, mode)) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(st, &cs);
+    if (cs != cudaStreamCaptureStatusNone)
+      return fail(h, MUON_ERR_INVALID_ARG,
+                  "a new list of shapes needs workspace set-up, which cannot run under stream capture");
+    if ((s = build_plan(h, rows, cols, n, mode, st))) return s;
+  }
+  const int final_buf = ns_steps & 1;
+  if ((s = launch_elementwise(h, cm, true, 0, 0, mu, nesterov, eps, st))) return s;
+  if ((s = launch_ns(h, coeffs, ns_steps, st))) return s;
+  if ((s = launch_elementwise(h, cm, false, step ? kEwApply : kEwExport, final_buf, mu, nesterov, eps, st)))
+    return s;
+  return finish_call(h, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+muon_status muon_init(muon_handle_t* out, int device) {
+  if (!out) return MUON_ERR_INVALID_ARG;
+  *out = nullptr;
+  int count = 0;
+  if (cudaGetDeviceCount(&count) != cudaSuccess) {
+    cudaGetLastError();
+    return MUON_ERR_CUDA;
+  }
+  if (device < 0 || device >= count) return MUON_ERR_INVALID_ARG;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return MUON_ERR_CUDA;
+  if (prop.major != 10 || prop.minor != 0) return MUON_ERR_UNSUPPORTED;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return MUON_ERR_CUDA;
+  muon_handle* h = new (std::nothrow) muon_handle();
+  if (!h) return MUON_ERR_OOM;
+  h->device = device;
+  h->sm_count = prop.multiProcessorCount;
+  h->encode = reinterpret_cast<EncodeTiledFn>(fn);
+  *out = h;
+  return MUON_OK;
+}
+
+muon_status muon_step(muon_handle_t h, const muon_matrix* mats, int n, float lr, float momentum, int nesterov,
+                      const float* coeffs, int ns_steps, float eps, muon_mode mode, void* cuda_stream) {
+  if (!h) return MUON_ERR_INVALID_ARG;
+  h->err.clear();
+  if (n < 0 || n > kMaxMatrices) return fail(h, MUON_ERR_INVALID_ARG, "n = %d outside 0..%d", n, kMaxMatrices);
+  if (n == 0) return MUON_OK;
+  if (!mats) return fail(h, MUON_ERR_INVALID_ARG, "mats is NULL");
+  if (!finite(lr) || lr < 0.f) return fail(h, MUON_ERR_INVALID_ARG, "lr must be finite and >= 0");
+  if (!finite(momentum) || momentum < 0.f || momentum >= 1.f)
+    return fail(h, MUON_ERR_INVALID_ARG, "momentum must lie in [0, 1)");
+  if (!finite(eps) || eps < 0.f) return fail(h, MUON_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (mode != MUON_MODE_BF16 && mode != MUON_MODE_FP32_VALIDATE)
+    return fail(h, MUON_ERR_INVALID_ARG, "unknown mode %d", (int)mode);
+  muon_status s = check_coeffs(h, coeffs, ns_steps);
+  if (s) return s;
+  std::vector<Range> ranges;
+  std::vector<int64_t> rows(n), cols(n);
+  std::vector<CallMat> cm(n);
+  for (int i = 0; i < n; ++i) {
+    const muon_matrix& m = mats[i];
+    if (!m.param || !m.grad || !m.momentum) return fail(h, MUON_ERR_INVALID_ARG, "matrix %d has a NULL pointer", i);
+    if (m.rows < 1 || m.cols < 1 || m.rows > kMaxDim || m.cols > kMaxDim)
+      return fail(h, MUON_ERR_INVALID_ARG, "matrix %d has shape %lld x %lld", i, (long long)m.rows,
+                  (long long)m.cols);
+    if ((m.param_dtype != MUON_F32 && m.param_dtype != MUON_BF16) ||
+        (m.grad_dtype != MUON_F32 && m.grad_dtype != MUON_BF16))
+      return fail(h, MUON_ERR_INVALID_ARG, "matrix %d has an unknown dtype", i);
+    if ((reinterpret_cast<uintptr_t>(m.param) | reinterpret_cast<uintptr_t>(m.grad) |
+         reinterpret_cast<uintptr_t>(m.momentum)) & 15u)
+      return fail(h, MUON_ERR_INVALID_ARG, "matrix %d has a pointer that is not 16-byte aligned", i);
+    const uint64_t numel = (uint64_t)m.rows * (uint64_t)m.cols;
+    const size_t pb = numel * (m.param_dtype == MUON_BF16 ? 2 : 4);
+    const size_t gb = numel * (m.grad_dtype == MUON_BF16 ? 2 : 4);
+    ranges.push_back({(uintptr_t)m.param, (uintptr_t)m.param + pb, i});
+    ranges.push_back({(uintptr_t)m.grad, (uintptr_t)m.grad + gb, i});
+    ranges.push_back({(uintptr_t)m.momentum, (uintptr_t)m.momentum + numel * 4, i});
+    rows[i] = m.rows;
+    cols[i] = m.cols;
+    const double scale = std::sqrt(std::max(1.0, (double)m.rows / (double)m.cols));
+    cm[i] = CallMat{m.param, m.grad, m.momentum, nullptr, m.param_dtype == MUON_BF16, m.grad_dtype == MUON_BF16,
+                    (float)((double)lr * scale)};
+  }
+  if ((s = check_overlaps(h, ranges))) return s;
+  return run(h, cm, rows.data(), cols.data(), true, momentum, nesterov ? 1 : 0, coeffs, ns_steps, eps, mode,
+             static_cast<cudaStream_t>(cuda_stream));
+}
+
+muon_status muon_newton_schulz(muon_handle_t h, const void* const* x_in, void* const* o_out, const int64_t* rows,
+                               const int64_t* cols, int n, muon_dtype dtype, const float* coeffs, int ns_steps,
+                               float eps, muon_mode mode, void* cuda_stream) {
+  if (!h) return MUON_ERR_INVALID_ARG;
+  h->err.clear();
+  if (n < 0 || n > kMaxMatrices) return fail(h, MUON_ERR_INVALID_ARG, "n = %d outside 0..%d", n, kMaxMatrices);
+  if (n == 0) return MUON_OK;
+  if (!x_in || !o_out || !rows || !cols) return fail(h, MUON_ERR_INVALID_ARG, "NULL array argument");
+  if (dtype != MUON_F32 && dtype != MUON_BF16) return fail(h, MUON_ERR_INVALID_ARG, "unknown dtype");
+  if (!finite(eps) || eps < 0.f) return fail(h, MUON_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (mode != MUON_MODE_BF16 && mode != MUON_MODE_FP32_VALIDATE)
+    return fail(h, MUON_ERR_INVALID_ARG, "unknown mode %d", (int)mode);
+  muon_status s = check_coeffs(h, coeffs, ns_steps);
+  if (s) return s;
+  std::vector<Range> ranges;
+  std::vector<CallMat> cm(n);
+  const size_t esz = dtype == MUON_BF16 ? 2 : 4;
+  for (int i = 0; i < n; ++i) {
+    if (!x_in[i] || !o_out[i]) return fail(h, MUON_ERR_INVALID_ARG, "matrix %d has a NULL pointer", i);
+    if (rows[i] < 1 || cols[i] < 1 || rows[i] > kMaxDim || cols[i] > kMaxDim)
+      return fail(h, MUON_ERR_INVALID_ARG, "matrix %d has shape %lld x %lld", i, (long long)rows[i],
+                  (long long)cols[i]);
+    if ((reinterpret_cast<uintptr_t>(x_in[i]) | reinterpret_cast<uintptr_t>(o_out[i])) & 15u)
+      return fail(h, MUON_ERR_INVALID_ARG, "matrix %d has a pointer that is not 16-byte aligned", i);
+    const size_t bytes = (size_t)rows[i] * (size_t)cols[i] * esz;
+    ranges.push_back({(uintptr_t)o_out[i], (uintptr_t)o_out[i] + bytes, i});
+    cm[i] = CallMat{const_cast<void*>(x_in[i]), nullptr, nullptr, o_out[i], dtype == MUON_BF16, false, 0.f};
+  }
+  if ((s = check_overlaps(h, ranges))) return s;
+  // outputs must not overlap any input either
+  for (int i = 0; i < n; ++i) {
+    const uintptr_t lo = (uintptr_t)x_in[i], hi = lo + (size_t)rows[i] * (size_t)cols[i] * esz;
+    for (const Range& r : ranges)
+      if (lo < r.hi && r.lo < hi)
+        return fail(h, MUON_ERR_INVALID_ARG, "output of matrix %d overlaps input of matrix %d", r.mat, i);
+  }
+  return run(h, cm, rows, cols, false, 0.f, 0, coeffs, ns_steps, eps, mode, static_cast<cudaStream_t>(cuda_stream));
+}
+
+muon_status muon_sync(muon_handle_t h) {
+  if (!h) return MUON_ERR_INVALID_ARG;
+  DeviceGuard dg(h->device);
+  return poll_status(h, true);
+}
+
+int64_t muon_workspace_bytes(muon_handle_t h) { return h ? (int64_t)h->ws_bytes : 0; }
+
+int muon_last_launch_count(muon_handle_t h) { return h ? h->last_launches : 0; }
+
+muon_status muon_destroy(muon_handle_t h) {
+  if (!h) return MUON_OK;
+  muon_status s = MUON_OK;
+  {
+    DeviceGuard dg(h->device);
+    s = poll_status(h, true);
+    if (h->ws) cudaFree(h->ws);
+    if (h->dev_status) cudaFree(h->dev_status);
+    if (h->host_status) cudaFreeHost(h->host_status);
+    if (h->status_event) cudaEventDestroy(h->status_event);
+  }
+  delete h;
+  return s;
+}
+
+const char* muon_status_string(muon_status s) {
+  switch (s) {
+    case MUON_OK: return "MUON_OK";
+    case MUON_ERR_INVALID_ARG: return "MUON_ERR_INVALID_ARG: invalid argument";
+    case MUON_ERR_UNSUPPORTED: return "MUON_ERR_UNSUPPORTED: unsupported device or combination";
+    case MUON_ERR_OOM: return "MUON_ERR_OOM: device allocation failed";
+    case MUON_ERR_CUDA: return "MUON_ERR_CUDA: CUDA call failed";
+    case MUON_ERR_TIMEOUT: return "MUON_ERR_TIMEOUT: a device-side wait timed out";
+    default: return "unknown muon_status";
+  }
+}
+
+const char* muon_last_error(muon_handle_t h) { return h ? h->err.c_str() : ""; }
+
+}  // extern "C"

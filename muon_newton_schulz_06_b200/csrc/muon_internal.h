@@ -1,0 +1,123 @@
+// Internal structures shared by the host driver (muon_api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace muon {
+
+// Device-side status codes written into the handle's status word.
+enum DevStatus : int {
+  kDevOk = 0,
+  kDevTimeout = 1,
+};
+
+// ----------------------------------------------------------------- elementwise passes
+
+// Max matrices handled by one elementwise launch (they travel as kernel
+// parameters; larger lists are split into several launches).
+constexpr int kMaxMatsPerLaunch = 192;
+
+// Square tile of one elementwise work unit.
+constexpr int kEwTile = 64;
+
+struct EwMat {
+  void* param;          // caller matrix: param (apply), or x_in (normalise-only)
+  const void* grad;     // caller gradient (momentum pass) / unused
+  float* mom;           // caller momentum buffer (momentum pass) / unused
+  void* work;           // workspace matrix in wide orientation, s x ld
+  int32_t rows, cols;   // caller shape
+  int32_t ld;           // leading dimension of the workspace matrix (elements)
+  int32_t tiles_c;      // number of 64-wide tile columns of the caller matrix
+  int32_t unit_begin;   // first work unit of this matrix inside the launch
+  int32_t gid;          // global matrix index (partials, counters, scales)
+  int32_t part_base;    // first norm partial of this matrix
+  int32_t n_units;      // work units of this matrix (= its norm partials)
+  uint8_t transposed;   // rows > cols: the workspace holds the transpose
+  uint8_t vec_ok;       // caller rows are 16-byte aligned: vector path allowed
+  uint8_t param_bf16;   // dtype of `param` (apply / export / normalise input)
+  uint8_t grad_bf16;    // dtype of `grad`
+  float lrs;            // fl32(lr * sqrt(max(1, rows/cols))) (apply)
+};
+
+struct EwParams {
+  EwMat mats[kMaxMatsPerLaunch];
+  int n_mats;
+  int total_units;
+  float mu;
+  int nesterov;
+  int use_momentum;     // 0: U = x_in (Newton-Schulz entry point)
+  float eps;
+  float* partials;      // per-unit sum of squares
+  unsigned* counters;   // per-matrix completed units (zero between launches)
+  float* scale;         // per-matrix 1/(||U||_F + eps)
+};
+
+enum EwOut : int { kEwApply = 0, kEwExport = 1 };
+
+// Launchers (k_elementwise.cu).  work_f32 selects the workspace element type.
+cudaError_t launch_momentum_norm(const EwParams& p, bool work_f32, int grid, cudaStream_t st);
+cudaError_t launch_apply(const EwParams& p, bool work_f32, int out_kind, int grid, cudaStream_t st);
+
+// ----------------------------------------------------------------- tensor-core engine
+
+// Shape groups per tensor-core launch (tensor maps travel as kernel parameters).
+constexpr int kMaxGroups = 12;
+
+constexpr int kBM = 128;   // tile rows (UMMA M)
+constexpr int kBN = 256;   // tile cols (UMMA N)
+constexpr int kBK = 64;    // k-block (one 128-byte swizzle row of bf16)
+
+enum TcPhase : int { kPhaseGram = 0, kPhasePoly = 1, kPhaseUpdate = 2 };
+
+struct TcTile {
+  uint16_t group;
+  uint16_t mat;   // index inside the group
+  uint16_t bi;    // 128-row block
+  uint16_t bj;    // 256-col block
+};
+
+struct TcGroup {
+  int s, L;              // matrix in wide orientation: s x L
+  int ld_x;              // leading dimension of X buffers (elements)
+  int ld_s;              // leading dimension of the s x s buffers
+  int gid_base;          // global index of matrix 0 of the group
+  __nv_bfloat16* x_cur;  // [n][s][ld_x]
+  __nv_bfloat16* x_next; // [n][s][ld_x]
+  __nv_bfloat16* gram;   // [n][s][ld_s]
+  __nv_bfloat16* poly;   // [n][s][ld_s]
+};
+
+struct __align__(64) TcParams {
+  CUtensorMap map_a[kMaxGroups];  // A operand (K-major, box 64 x 128)
+  CUtensorMap map_b[kMaxGroups];  // B operand (K-major box 64 x 128, or MN-major box 64 x 64)
+  TcGroup g[kMaxGroups];
+  const TcTile* tiles;
+  int n_tiles;
+  int first_iter;                 // fold the Frobenius scale into this pass
+  float ca, cb, cc;               // coefficient triple of this step
+  const float* scale;             // per-matrix 1/(||U||_F + eps)
+  int* status;                    // device status word
+};
+
+cudaError_t launch_tc(int phase, const TcParams& p, int grid, cudaStream_t st);
+int tc_smem_bytes();
+
+// ----------------------------------------------------------------- fp32 validation path
+
+struct F32Mat {
+  float* x_cur;
+  float* x_next;
+  float* gram;
+  float* poly;
+  int s, L, ld_x, ld_s, gid;
+};
+
+cudaError_t launch_f32_gram(const F32Mat& m, int first_iter, const float* scale, cudaStream_t st);
+cudaError_t launch_f32_poly(const F32Mat& m, float cb, float cc, cudaStream_t st);
+cudaError_t launch_f32_update(const F32Mat& m, int first_iter, const float* scale, float ca,
+                              cudaStream_t st);
+
+}  // namespace muon

@@ -1,0 +1,272 @@
+"""CUDA path vs the CPU oracle, through the C ABI (the Python binding only marshals
+arguments).  Needs a B200.
+
+Tolerances (relative Frobenius error of the orthogonalised update per matrix):
+bf16 mode 2e-2, fp32 validation mode 1e-4; momentum buffers bit-exact.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+BF16_TOL = 2e-2
+F32_TOL = 1e-4
+
+
+@pytest.fixture(scope="module")
+def mb():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import muon_newton_schulz_06_b200 as m
+    from muon_newton_schulz_06_b200 import build
+    build.build()
+    return m
+
+
+@pytest.fixture(scope="module")
+def handle(mb):
+    h = mb.muon_init(0)
+    yield h
+    mb.muon_destroy(h)
+
+
+def rel(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def to64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def ns_gpu(mb, handle, xs, mode, coeffs=None, ns_steps=5, eps=1e-7):
+    outs = [torch.empty_like(x) for x in xs]
+    mb.muon_newton_schulz(handle, xs, outs, coeffs=coeffs, ns_steps=ns_steps, eps=eps, mode=mode)
+    torch.cuda.synchronize()
+    mb.muon_sync(handle)
+    return outs
+
+
+def ns_oracle(x, coeffs, eps=1e-7):
+    return oracle.newton_schulz(oracle.frobenius_normalise(to64(x), eps), coeffs)
+
+
+EDGE_SHAPES = [(1, 9), (9, 1), (1, 1), (63, 130), (130, 63), (64, 64), (65, 257), (257, 65), (129, 129),
+               (127, 300), (300, 255), (96, 96), (256, 32), (384, 1000)]
+
+
+# ------------------------------------------------------------- single Newton-Schulz step algebra
+
+@pytest.mark.parametrize("mode,dtype,tol", [("fp32", torch.float32, 1e-5), ("bf16", torch.bfloat16, 1.5e-2)])
+@pytest.mark.parametrize("abc", [(1.0, 0.0, 0.0), (0.0, 1.0, 0.0), (0.0, 0.0, 1.0), (0.5, -1.0, 2.0)])
+def test_one_step_each_product(mb, handle, mode, dtype, tol, abc):
+    """(1,0,0) passes X through; (0,1,0) is X X^T X (Gram + update); (0,0,1) is (X X^T)^2 X
+    (Gram + polynomial + update)."""
+    shapes = [(200, 136), (136, 200), (256, 512), (130, 130), (40, 700)]
+    xs = [synth.random_matrix(r, c, seed=10 + i, device="cuda", dtype=dtype) for i, (r, c) in enumerate(shapes)]
+    outs = ns_gpu(mb, handle, xs, mode, coeffs=[abc], ns_steps=1)
+    for x, o in zip(xs, outs):
+        want = ns_oracle(x, [abc])
+        assert rel(to64(o), want) < tol, (x.shape, abc, rel(to64(o), want))
+
+
+# ------------------------------------------------------------- full Newton-Schulz
+
+@pytest.mark.parametrize("mode,dtype,tol", [("fp32", torch.float32, F32_TOL), ("bf16", torch.bfloat16, BF16_TOL)])
+def test_newton_schulz_edge_shapes(mb, handle, mode, dtype, tol):
+    """Shapes around the 64 / 128 / 256 tile edges, tall, wide, square and degenerate,
+    all in one grouped call.  Inputs are well conditioned (singular values in
+    [0.05, 1]) so the comparison measures the kernels, not the input rounding."""
+    xs = []
+    for i, (r, c) in enumerate(EDGE_SHAPES):
+        g = torch.Generator().manual_seed(500 + i)
+        k = min(r, c)
+        u, _ = torch.linalg.qr(torch.randn(r, k, generator=g, dtype=torch.float64))
+        v, _ = torch.linalg.qr(torch.randn(c, k, generator=g, dtype=torch.float64))
+        s = 0.05 + 0.95 * torch.rand(k, generator=g, dtype=torch.float64)
+        xs.append(((u * s) @ v.T).to(dtype).cuda().contiguous())
+    outs = ns_gpu(mb, handle, xs, mode)
+    for x, o in zip(xs, outs):
+        want = ns_oracle(x, [oracle.QUINTIC] * 5)
+        err = rel(to64(o), want)
+        assert err < tol, (tuple(x.shape), err)
+
+
+def test_newton_schulz_gaussian_bf16(mb, handle):
+    """Gaussian inputs (tiny singular values included) at the 2e-2 bar."""
+    shapes = [(512, 512), (2048, 512), (512, 2048), (768, 768)]
+    xs = [synth.random_matrix(r, c, seed=70 + i, device="cuda", dtype=torch.bfloat16) for i, (r, c) in
+          enumerate(shapes)]
+    outs = ns_gpu(mb, handle, xs, "bf16")
+    for x, o in zip(xs, outs):
+        err = rel(to64(o), ns_oracle(x, [oracle.QUINTIC] * 5))
+        assert err < BF16_TOL, (tuple(x.shape), err)
+
+
+def test_transpose_equivariance_gpu(mb, handle):
+    x = synth.random_matrix(300, 130, seed=3, device="cuda", dtype=torch.bfloat16)
+    xt = x.T.contiguous()
+    o, ot = ns_gpu(mb, handle, [x, xt], "bf16")
+    # both orientations run the same kernels on the same wide-orientation data; only the
+    # norm's summation order differs
+    assert rel(to64(o).T, to64(ot)) < 1e-2
+
+
+# ------------------------------------------------------------- whole step, tiny set
+
+@pytest.mark.parametrize("mode,tol", [("fp32", F32_TOL), ("bf16", BF16_TOL)])
+def test_tiny_set_three_steps(mb, handle, mode, tol):
+    """Tiny set: 128x64, 64x128, 96x96, 256x32, fp32, N(0,1) grads, M = W = 0, mu 0.95
+    Nesterov, lr 0.02, quintic x5, eps 1e-7, three steps with the same gradient."""
+    data = synth.make_matrix_set(0)
+    W = [w.cuda() for w in data["W"]]
+    G = [g.cuda() for g in data["G"]]
+    M = [m.cuda() for m in data["M"]]
+    ow = [to64(w) for w in data["W"]]
+    om = [m.numpy() for m in data["M"]]
+    for step in range(3):
+        prev = [to64(w) for w in W]
+        mb.muon_step(handle, W, G, M, lr=0.02, momentum=0.95, nesterov=True, mode=mode)
+        torch.cuda.synchronize()
+        mb.muon_sync(handle)
+        for i, spec in enumerate(data["specs"]):
+            w_new, m_new, o = oracle.muon_step_matrix(ow[i], data["G"][i].numpy(), om[i], lr=0.02, mu=0.95,
+                                                      nesterov=True, eps=1e-7)
+            # momentum: bit-exact
+            assert np.array_equal(M[i].cpu().numpy(), m_new), (step, spec)
+            # update: W_new - W_prev vs -lr*scale*O
+            dw = to64(W[i]) - prev[i]
+            err = rel(dw, w_new - ow[i])
+            assert err < tol, (step, spec, err)
+            ow[i], om[i] = w_new, m_new
+
+
+# ------------------------------------------------------------- apply exactness and momentum (bf16 sets)
+
+def test_apply_exact_and_momentum_bitexact(mb, handle):
+    """With fp32 zero weights and lr = 1, W' = -fl32(scale*O) is exact for scale in {1, 2}, so
+    O is read back; a second run from the same state with bf16 weights must give
+    RNE(fl32(W - fl32(lr*scale)*O)) bit for bit.  Momentum vs NumPy float32, bit for bit."""
+    data = synth.make_matrix_set(1, layers=[0, 1])
+    G = [g.cuda() for g in data["G"]]
+    M0 = [m.cuda() for m in data["M"]]
+    scales = [math.sqrt(max(1.0, s.rows / s.cols)) for s in data["specs"]]
+    assert set(scales) <= {1.0, 2.0}
+    # run 1: fp32 zeros, lr = 1
+    M = [m.clone() for m in M0]
+    Wz = [torch.zeros(s.rows, s.cols, device="cuda") for s in data["specs"]]
+    mb.muon_step(handle, Wz, G, M, lr=1.0, momentum=0.95, nesterov=True)
+    torch.cuda.synchronize()
+    mb.muon_sync(handle)
+    O = [(-w / sc) for w, sc in zip(Wz, scales)]
+    for i in range(len(G)):
+        m_ref, _ = oracle.nesterov_momentum_f32(data["G"][i].float().numpy(), data["M"][i].numpy(), 0.95, True)
+        assert np.array_equal(M[i].cpu().numpy(), m_ref)
+    # run 2: same state, bf16 weights
+    M = [m.clone() for m in M0]
+    W = [w.cuda().clone() for w in data["W"]]
+    W_before = [w.clone() for w in W]
+    lr = 0.02
+    mb.muon_step(handle, W, G, M, lr=lr, momentum=0.95, nesterov=True)
+    torch.cuda.synchronize()
+    for i in range(len(G)):
+        lrs = np.float32(lr * scales[i])
+        o = O[i].cpu().numpy().astype(np.float32)
+        want = np.subtract(W_before[i].float().cpu().numpy(), np.multiply(lrs, o, dtype=np.float32),
+                           dtype=np.float32)
+        want_bf16 = torch.from_numpy(want).to(torch.bfloat16)
+        assert torch.equal(W[i].cpu(), want_bf16), i
+    # and O itself is the oracle's within the bf16 bar
+    for i in range(len(G)):
+        _, _, o_ref = oracle.muon_step_matrix(np.zeros((data["specs"][i].rows, data["specs"][i].cols)),
+                                              data["G"][i].float().numpy(), data["M"][i].numpy(), lr=1.0,
+                                              mu=0.95, nesterov=True, eps=1e-7)
+        assert rel(to64(O[i]), o_ref) < BF16_TOL, i
+
+
+def test_grouped_step_matches_single_matrix_calls(mb, handle):
+    """Packing many shapes into one grouped launch gives the same bits as one call per matrix."""
+    data = synth.make_matrix_set(1, layers=[0])
+    G = [g.cuda() for g in data["G"]]
+    W1 = [w.cuda().clone() for w in data["W"]]
+    M1 = [m.cuda().clone() for m in data["M"]]
+    W2 = [w.clone() for w in W1]
+    M2 = [m.clone() for m in M1]
+    mb.muon_step(handle, W1, G, M1, lr=0.02)
+    h2 = mb.muon_init(0)
+    try:
+        for i in range(len(G)):
+            mb.muon_step(h2, [W2[i]], [G[i]], [M2[i]], lr=0.02)
+        torch.cuda.synchronize()
+    finally:
+        mb.muon_destroy(h2)
+    for a, b in zip(W1, W2):
+        assert torch.equal(a, b)
+    for a, b in zip(M1, M2):
+        assert torch.equal(a, b)
+
+
+def test_zero_gradient_leaves_weights(mb, handle):
+    W = [torch.randn(256, 128, device="cuda").to(torch.bfloat16), torch.randn(64, 300, device="cuda")]
+    G = [torch.zeros_like(w) for w in W]
+    M = [torch.zeros(w.shape, device="cuda") for w in W]
+    before = [w.clone() for w in W]
+    mb.muon_step(handle, W, G, M, lr=0.1)
+    torch.cuda.synchronize()
+    mb.muon_sync(handle)
+    for a, b in zip(W, before):
+        assert torch.equal(a, b)
+    for m in M:
+        assert torch.count_nonzero(m) == 0
+
+
+def test_nesterov_off(mb, handle):
+    data = synth.make_matrix_set(0)
+    W = [torch.zeros_like(w).cuda() for w in data["W"]]
+    G = [g.cuda() for g in data["G"]]
+    M = [(0.5 * g).cuda() for g in data["G"]]
+    mb.muon_step(handle, W, G, M, lr=1.0, momentum=0.9, nesterov=False, mode="fp32")
+    torch.cuda.synchronize()
+    for i, spec in enumerate(data["specs"]):
+        w_new, _, _ = oracle.muon_step_matrix(np.zeros((spec.rows, spec.cols)), data["G"][i].numpy(),
+                                              (0.5 * data["G"][i]).numpy(), lr=1.0, mu=0.9, nesterov=False)
+        assert rel(to64(W[i]), w_new) < F32_TOL
+
+
+# ------------------------------------------------------------- argument errors (host-side)
+
+def test_invalid_arguments(mb, handle):
+    w = torch.zeros(64, 64, device="cuda")
+    g = torch.zeros(64, 64, device="cuda")
+    m = torch.zeros(64, 64, device="cuda")
+    with pytest.raises(mb.MuonError) as e:
+        mb.muon_step(handle, [w], [g], [m], lr=float("nan"))
+    assert e.value.code == mb.MUON_ERR_INVALID_ARG
+    with pytest.raises(mb.MuonError):
+        mb.muon_step(handle, [w], [g], [m], lr=0.1, momentum=1.0)
+    with pytest.raises(mb.MuonError):
+        mb.muon_step(handle, [w], [g], [m], lr=0.1, ns_steps=0)
+    with pytest.raises(mb.MuonError):
+        mb.muon_step(handle, [w], [w], [m], lr=0.1)  # param aliases grad
+    with pytest.raises(mb.MuonError):
+        mb.muon_step(handle, [w, w], [g, g], [m, m], lr=0.1)
+    mis = torch.zeros(64 * 64 + 1, device="cuda")[1:].view(64, 64)
+    with pytest.raises(mb.MuonError) as e:
+        mb.muon_step(handle, [mis], [g], [m], lr=0.1)
+    assert e.value.code == mb.MUON_ERR_INVALID_ARG
+    # nothing was enqueued by the failed calls and the handle still works
+    mb.muon_step(handle, [w], [g], [m], lr=0.1)
+    torch.cuda.synchronize()
+    mb.muon_sync(handle)
+
+
+def test_empty_call_is_a_no_op(mb, handle):
+    mb.muon_step(handle, [], [], [], lr=0.1)
+    mb.muon_newton_schulz(handle, [], [])
