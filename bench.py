@@ -1,0 +1,367 @@
+#!/usr/bin/env python
+"""Benchmark of the Muon optimizer step on B200 (one process per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4] [--impl ours|reference]
+
+One step = one muon_step call over the whole matrix set of the workload: momentum +
+norm pass, five Newton-Schulz steps (Gram, polynomial, update launches) and the
+apply pass, on seeded synthetic gradients with the shapes of the 3.8B Llama-style
+model (168 matrices, 2.82B parameters; inputs larger than L2).  Rank 0 prints one
+JSON line.
+
+value      algorithmic Newton-Schulz TFLOP (one triangle of the symmetric products)
+           per step x steps, summed over ranks, / the slowest rank's device time of
+           the whole steps (CUDA events on the launch stream).
+e2e        the same metric when every step also copies the gradients in from pinned
+           host memory and the updated weights back out.
+roofline   the kernel with the largest share of device time, from per-launch CUDA
+           events the library records on its stream during the timed steps.
+cpu_baseline  the float64 CPU oracle on a bounded sample of the same workload.
+--gpus N>1 runs N independent replicas of the full set (weak scaling): the step has no
+data exchange, so there is no collective on the data path.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Muon step ms & NS TFLOP/s (fraction of bf16 tensor peak) per model matrix set, 1 B200"
+UNIT = "TFLOP/s"
+LR, MU, EPS, NS_STEPS = 0.02, 0.95, 1e-7, 5
+WORKLOAD_TEXT = {
+    1: "d8: depth-8 GPT, d_model 512, MLP 2048, 48 bf16 matrices",
+    2: "d12: depth-12 GPT, d_model 768, MLP 3072, 72 bf16 matrices",
+    3: "d24: depth-24 GPT, d_model 1536, MLP 6144, 144 bf16 matrices, heavy-tailed gradient spectrum",
+    4: ("llama3p8b: 168 matrices of the 3.8B Llama-style model (28 layers: Wq 3072x3072, Wk/Wv 1024x3072, "
+        "Wo 3072x3072, W_fc 12288x3072, W_proj 3072x12288), bf16 params and grads, fp32 momentum"),
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=4, choices=[1, 2, 3, 4])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks during the timed region
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.gpu_id:
+            cmd.insert(1, f"--id={self.gpu_id}")
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def oracle_sample(config, seconds, device_data=None):
+    """Times the float64 oracle step on matrices of layer 0 (then further layers) of the
+    workload until `seconds` of CPU time have passed.  Returns (flops, time, names, cores)."""
+    import numpy as np
+
+    import oracle
+    import synth
+    from muon_newton_schulz_06_b200 import cost
+
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info() if i.get("user_api") == "blas"] or [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    specs = synth.config_shapes(config)
+    flops, spent, names = 0, 0.0, []
+    for idx, spec in enumerate(specs):
+        if device_data is not None and idx < len(device_data["G"]):
+            g = device_data["G"][idx].float().cpu().numpy()
+            m = device_data["M"][idx].cpu().numpy()
+            w = device_data["W"][idx].float().cpu().numpy()
+        else:
+            d = synth.make_matrix_set(config, device="cpu", indices=[idx])
+            g, m, w = d["G"][0].float().numpy(), d["M"][0].numpy(), d["W"][0].float().numpy()
+        t0 = time.perf_counter()
+        oracle.muon_step_matrix(w.astype(np.float64), g, m, lr=LR, mu=MU, nesterov=True, eps=EPS)
+        spent += time.perf_counter() - t0
+        flops += cost.ns_flops([(spec.rows, spec.cols)], NS_STEPS)["algorithmic"]
+        names.append(spec.name)
+        if spent >= seconds:
+            break
+    return flops, spent, names, cores
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import synth
+    from muon_newton_schulz_06_b200 import cost
+    cfg = args.config
+    # each step: the oracle on one Wk-shaped matrix of layer 0 (a bounded sample of the set)
+    specs = synth.config_shapes(cfg)
+    pick = min(range(len(specs)), key=lambda i: specs[i].rows * specs[i].cols)
+    import numpy as np
+
+    import oracle
+    d = synth.make_matrix_set(cfg, device="cpu", indices=[pick])
+    g, m, w = d["G"][0].float().numpy(), d["M"][0].numpy(), d["W"][0].float().numpy().astype(np.float64)
+    for _ in range(args.warmup):
+        oracle.muon_step_matrix(w, g, m, lr=LR, mu=MU, nesterov=True, eps=EPS)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        w, m, _ = oracle.muon_step_matrix(w, g, m, lr=LR, mu=MU, nesterov=True, eps=EPS)
+    dt = time.perf_counter() - t0
+    spec = specs[pick]
+    flops = cost.ns_flops([(spec.rows, spec.cols)], NS_STEPS)["algorithmic"] * args.steps
+    value = flops / dt / 1e12
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info() if i.get("user_api") == "blas"] or [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    sample = f"one {spec.rows}x{spec.cols} matrix ({spec.name}) of the set per step, float64 NumPy oracle"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD_TEXT[cfg], "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    import muon_newton_schulz_06_b200 as mb
+    import synth
+    from muon_newton_schulz_06_b200 import cost
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    cfg = args.config
+    data = synth.make_matrix_set(cfg, device=dev)
+    W, G, M = data["W"], data["G"], data["M"]
+    shapes = [(s.rows, s.cols) for s in data["specs"]]
+    fl = cost.ns_flops(shapes, NS_STEPS)
+    eb = cost.elementwise_bytes(shapes)
+    torch.cuda.synchronize()
+
+    h = mb.muon_init(local)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mb.muon_step(h, W, G, M, lr=LR, momentum=MU, nesterov=True, ns_steps=NS_STEPS, eps=EPS, stream=stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    mb.muon_sync(h)
+    launches_per_step = mb.muon_last_launch_count(h)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---------------- device-timed region
+    mb.muon_profile_enable(h, True)
+    mb.muon_profile_read(h)
+    gpu_uuid = None
+    try:
+        gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if gpu_uuid and not gpu_uuid.startswith("GPU-"):
+            gpu_uuid = "GPU-" + gpu_uuid
+    except Exception:
+        gpu_uuid = None
+    sampler = ClockSampler(gpu_uuid)
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    mb.muon_sync(h)
+    ms = e0.elapsed_time(e1)
+    prof = mb.muon_profile_read(h)
+    mb.muon_profile_enable(h, False)
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    value = fl["algorithmic"] * args.steps * world / (ms_max / 1e3) / 1e12
+
+    # ---------------- end to end: pinned host gradients in, updated weights out, every step
+    e2e = None
+    if not args.no_e2e:
+        g_host = [g.cpu().pin_memory() for g in G]
+        w_host = [torch.empty(w.shape, dtype=w.dtype, pin_memory=True) for w in W]
+        h2d = sum(x.numel() * x.element_size() for x in g_host)
+        d2h = sum(x.numel() * x.element_size() for x in w_host)
+        e2 = torch.cuda.Event(enable_timing=True)
+        e3 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e2.record(stream)
+        for _ in range(args.steps):
+            for gd, gh in zip(G, g_host):
+                gd.copy_(gh, non_blocking=True)
+            step()
+            for wd, wh in zip(W, w_host):
+                wh.copy_(wd, non_blocking=True)
+        e3.record(stream)
+        torch.cuda.synchronize()
+        t2 = torch.tensor([e2.elapsed_time(e3)], device=dev, dtype=torch.float64)
+        if world > 1:
+            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t2.item())
+        e2e = {"value": fl["algorithmic"] * args.steps * world / (ms_e2e / 1e3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / args.steps}
+        del g_host, w_host
+
+    # ---------------- per-kernel roofline
+    pk = peaks()
+    kernels = {}
+    for kind, (kms, n) in prof.items():
+        if n == 0:
+            continue
+        avg_ms = kms / n
+        if kind in ("gram", "poly", "update"):
+            work = fl["per_launch"][kind]
+            ach = work / (avg_ms / 1e3) / 1e12
+            kernels[kind] = {"bound": "tensor", "ms_per_launch": avg_ms, "launches": n, "achieved": ach,
+                             "unit": "TFLOP/s", "work_per_launch": work,
+                             "frac": ach / pk["bf16_tflops_sustained"]}
+        else:
+            work = eb[kind]
+            ach = work / (avg_ms / 1e3) / 1e9
+            kernels[kind] = {"bound": "hbm", "ms_per_launch": avg_ms, "launches": n, "achieved": ach,
+                             "unit": "GB/s", "work_per_launch": work, "frac": ach / pk["hbm_gbs"]}
+        kernels[kind]["share"] = kms / max(sum(v[0] for v in prof.values()), 1e-9)
+    dom = max(kernels, key=lambda k: kernels[k]["share"])
+    dk = kernels[dom]
+    roofline = {"bound": dk["bound"], "kernel": dom, "achieved": dk["achieved"],
+                "peak": pk["bf16_tflops_sustained"] if dk["bound"] == "tensor" else pk["hbm_gbs"],
+                "peak_kind": ("sustained bf16 (kernel timed inside a long loop), " if dk["bound"] == "tensor"
+                              else "copy bandwidth, ") + pk["source"],
+                "unit": dk["unit"], "frac": dk["frac"], "traffic": None}
+    ns_ms = sum(prof[k][0] for k in ("gram", "poly", "update")) / args.steps
+    ns_tflops = fl["algorithmic"] / (ns_ms / 1e3) / 1e12 if ns_ms > 0 else None
+
+    # ---------------- CPU oracle on a bounded sample (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        flops_s, secs, names, cores = oracle_sample(cfg, args.cpu_sample_seconds, data)
+        cpu = {"value": flops_s / secs / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"float64 NumPy oracle step on {len(names)} matrices of the set ({', '.join(names)}), "
+                         f"{secs:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD_TEXT[cfg], "matrices": len(shapes),
+                       "params": int(eb["numel"]), "ns_steps": NS_STEPS,
+                       "coeffs": "quintic (3.4445, -4.7750, 2.0315) every step", "lr": LR, "momentum": MU,
+                       "nesterov": True, "eps": EPS,
+                       "l2": "no flush: inputs larger than L2 (%.1f GB of gradients per step)" % (
+                           sum(g.numel() * g.element_size() for g in G) / 1e9),
+                       "parallelism": "replicas" if world > 1 else "single GPU"},
+            "ns_tflops_algorithmic": ns_tflops,
+            "ns_frac_of_sustained_peak": ns_tflops / pk["bf16_tflops_sustained"] if ns_tflops else None,
+            "ns_frac_of_burst_peak": ns_tflops / pk["bf16_tflops"] if ns_tflops else None,
+            "ns_tflop_per_step_algorithmic": fl["algorithmic"] / 1e12,
+            "ns_tflop_per_step_dense_equivalent": fl["dense_equivalent"] / 1e12,
+            "matrices_per_s": len(shapes) * args.steps * world / (ms_max / 1e3),
+            "kernels": kernels, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    mb.muon_destroy(h)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

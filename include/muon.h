@@ -130,6 +130,27 @@ MUON_API int64_t muon_workspace_bytes(muon_handle_t h);
 /* Number of kernel launches the last muon_step / muon_newton_schulz enqueued. */
 MUON_API int muon_last_launch_count(muon_handle_t h);
 
+/* Kernel kinds reported by muon_profile_read. */
+typedef enum {
+  MUON_KIND_MOMENTUM_NORM = 0,  /* momentum + Nesterov + Frobenius norm pass */
+  MUON_KIND_GRAM = 1,           /* A = X X^T (scaled) */
+  MUON_KIND_POLY = 2,           /* B = b A + c A^2 */
+  MUON_KIND_UPDATE = 3,         /* X' = a X + B X */
+  MUON_KIND_APPLY = 4,          /* W -= lr*scale*O, or the export of O */
+  MUON_KIND_COUNT = 5
+} muon_kernel_kind;
+
+/* Per-launch timing: while enabled, every launch of the handle is bracketed by two
+ * CUDA events recorded on the launch stream.  Adds two event records per launch; no
+ * effect on results. */
+MUON_API muon_status muon_profile_enable(muon_handle_t h, int enable);
+
+/* Waits for the recorded events and writes, per kernel kind (indexed by
+ * muon_kernel_kind, arrays of length MUON_KIND_COUNT), the summed device time in
+ * milliseconds and the number of launches since the last read; then resets the
+ * totals.  ms and launches are HOST arrays. */
+MUON_API muon_status muon_profile_read(muon_handle_t h, double* ms, int64_t* launches);
+
 /* Waits for outstanding work, frees the workspace and the handle.  Returns the
  * pending device-side status.  NULL is accepted and returns MUON_OK. */
 MUON_API muon_status muon_destroy(muon_handle_t h);

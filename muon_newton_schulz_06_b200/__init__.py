@@ -32,7 +32,11 @@ MUON_MODE_BF16 = 0
 MUON_MODE_FP32_VALIDATE = 1
 
 EXPORTED = ("muon_init", "muon_step", "muon_newton_schulz", "muon_sync", "muon_workspace_bytes",
-            "muon_last_launch_count", "muon_destroy", "muon_status_string", "muon_last_error")
+            "muon_last_launch_count", "muon_profile_enable", "muon_profile_read", "muon_destroy",
+            "muon_status_string", "muon_last_error")
+
+# muon_kernel_kind
+KERNEL_KINDS = ("momentum_norm", "gram", "poly", "update", "apply")
 
 
 class MuonError(RuntimeError):
@@ -73,6 +77,10 @@ def load_library(path: str = LIB_PATH):
     lib.muon_workspace_bytes.restype = i64
     lib.muon_last_launch_count.argtypes = [vp]
     lib.muon_last_launch_count.restype = i32
+    lib.muon_profile_enable.argtypes = [vp, i32]
+    lib.muon_profile_enable.restype = i32
+    lib.muon_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)]
+    lib.muon_profile_read.restype = i32
     lib.muon_destroy.argtypes = [vp]
     lib.muon_destroy.restype = i32
     lib.muon_status_string.argtypes = [i32]
@@ -201,6 +209,19 @@ def muon_workspace_bytes(handle) -> int:
 
 def muon_last_launch_count(handle) -> int:
     return int(load_library().muon_last_launch_count(handle))
+
+
+def muon_profile_enable(handle, enable: bool = True) -> None:
+    _check(load_library().muon_profile_enable(handle, 1 if enable else 0), handle)
+
+
+def muon_profile_read(handle) -> dict:
+    """{kind: (total_ms, launches)} since the last read (waits for the recorded events)."""
+    n = len(KERNEL_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
+    _check(load_library().muon_profile_read(handle, ms, cnt), handle)
+    return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(KERNEL_KINDS)}
 
 
 def muon_destroy(handle) -> None:

@@ -84,6 +84,17 @@ struct muon_handle {
   cudaEvent_t status_event = nullptr;
   bool status_pending = false;
   Plan plan;
+  // per-launch timing (muon_profile_enable)
+  bool profiling = false;
+  std::vector<cudaEvent_t> ev_free;
+  struct Pending {
+    int kind;
+    cudaEvent_t a, b;
+  };
+  std::vector<Pending> ev_pending;
+  cudaEvent_t ev_open = nullptr;
+  double prof_ms[MUON_KIND_COUNT] = {};
+  int64_t prof_launches[MUON_KIND_COUNT] = {};
 };
 
 namespace {
@@ -102,6 +113,36 @@ muon_status fail(muon_handle* h, muon_status st, const char* fmt, ...) {
 
 muon_status cuda_fail(muon_handle* h, cudaError_t e, const char* what) {
   return fail(h, MUON_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+cudaEvent_t take_event(muon_handle* h) {
+  if (!h->ev_free.empty()) {
+    cudaEvent_t e = h->ev_free.back();
+    h->ev_free.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return e;
+}
+
+// Brackets one launch with events on its stream while profiling is on.
+void prof_begin(muon_handle* h, cudaStream_t st) {
+  if (!h->profiling) return;
+  h->ev_open = take_event(h);
+  if (h->ev_open) cudaEventRecord(h->ev_open, st);
+}
+
+void prof_end(muon_handle* h, int kind, cudaStream_t st) {
+  if (!h->profiling || !h->ev_open) return;
+  cudaEvent_t b = take_event(h);
+  if (!b) return;
+  cudaEventRecord(b, st);
+  h->ev_pending.push_back({kind, h->ev_open, b});
+  h->ev_open = nullptr;
 }
 
 // Restores the caller's current device on scope exit.
@@ -372,8 +413,10 @@ muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, b
     }
     ep->total_units = units;
     const int grid = std::max(1, std::min(units, h->sm_count * 8));
+    prof_begin(h, st);
     cudaError_t err = momentum_pass ? launch_momentum_norm(*ep, f32, grid, st)
                                     : launch_apply(*ep, f32, out_kind, grid, st);
+    prof_end(h, momentum_pass ? MUON_KIND_MOMENTUM_NORM : MUON_KIND_APPLY, st);
     delete ep;
     if (err != cudaSuccess) return cuda_fail(h, err, momentum_pass ? "momentum/norm launch" : "apply launch");
     h->last_launches++;
@@ -397,9 +440,15 @@ muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, cudaStr
         f.gram = reinterpret_cast<float*>(h->ws + g.off_gram + (size_t)m.idx * g.s * g.ld_s * 4);
         f.poly = reinterpret_cast<float*>(h->ws + g.off_poly + (size_t)m.idx * g.s * g.ld_s * 4);
         f.s = g.s; f.L = g.L; f.ld_x = g.ld_x; f.ld_s = g.ld_s; f.gid = g.gid_base + m.idx;
+        prof_begin(h, st);
         cudaError_t e = launch_f32_gram(f, k == 0, scale, st);
+        prof_end(h, MUON_KIND_GRAM, st);
+        prof_begin(h, st);
         if (e == cudaSuccess) e = launch_f32_poly(f, c[1], c[2], st);
+        prof_end(h, MUON_KIND_POLY, st);
+        prof_begin(h, st);
         if (e == cudaSuccess) e = launch_f32_update(f, k == 0, scale, c[0], st);
+        prof_end(h, MUON_KIND_UPDATE, st);
         if (e != cudaSuccess) return cuda_fail(h, e, "fp32 Newton-Schulz launch");
         h->last_launches += 3;
       }
@@ -440,7 +489,9 @@ muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, cudaStr
         tp->scale = scale;
         tp->status = h->dev_status;
         const int grid = std::max(1, std::min(tp->n_tiles, h->sm_count));
+        prof_begin(h, st);
         cudaError_t e = launch_tc(ph, *tp, grid, st);
+        prof_end(h, MUON_KIND_GRAM + ph, st);
         if (e != cudaSuccess) {
           delete tp;
           return cuda_fail(h, e, "tensor-core Newton-Schulz launch");
@@ -643,6 +694,39 @@ muon_status muon_sync(muon_handle_t h) {
   return poll_status(h, true);
 }
 
+muon_status muon_profile_enable(muon_handle_t h, int enable) {
+  if (!h) return MUON_ERR_INVALID_ARG;
+  h->profiling = enable != 0;
+  return MUON_OK;
+}
+
+muon_status muon_profile_read(muon_handle_t h, double* ms, int64_t* launches) {
+  if (!h || !ms || !launches) return MUON_ERR_INVALID_ARG;
+  DeviceGuard dg(h->device);
+  muon_status st = MUON_OK;
+  for (auto& p : h->ev_pending) {
+    float t = 0.f;
+    cudaError_t e = cudaEventSynchronize(p.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, p.a, p.b);
+    if (e != cudaSuccess) {
+      st = cuda_fail(h, e, "profile event");
+    } else {
+      h->prof_ms[p.kind] += t;
+      h->prof_launches[p.kind] += 1;
+    }
+    h->ev_free.push_back(p.a);
+    h->ev_free.push_back(p.b);
+  }
+  h->ev_pending.clear();
+  for (int k = 0; k < MUON_KIND_COUNT; ++k) {
+    ms[k] = h->prof_ms[k];
+    launches[k] = h->prof_launches[k];
+    h->prof_ms[k] = 0.0;
+    h->prof_launches[k] = 0;
+  }
+  return st;
+}
+
 int64_t muon_workspace_bytes(muon_handle_t h) { return h ? (int64_t)h->ws_bytes : 0; }
 
 int muon_last_launch_count(muon_handle_t h) { return h ? h->last_launches : 0; }
@@ -657,6 +741,11 @@ muon_status muon_destroy(muon_handle_t h) {
     if (h->dev_status) cudaFree(h->dev_status);
     if (h->host_status) cudaFreeHost(h->host_status);
     if (h->status_event) cudaEventDestroy(h->status_event);
+    for (auto& p : h->ev_pending) {
+      cudaEventDestroy(p.a);
+      cudaEventDestroy(p.b);
+    }
+    for (cudaEvent_t e : h->ev_free) cudaEventDestroy(e);
   }
   delete h;
   return s;
