@@ -63,7 +63,8 @@ typedef enum {
   MUON_ERR_UNSUPPORTED = 2,  /* a combination this build does not implement (e.g. no sm_100 device) */
   MUON_ERR_OOM = 3,          /* workspace allocation failed */
   MUON_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed */
-  MUON_ERR_TIMEOUT = 5       /* a bounded device-side wait expired (kernel gave up and returned) */
+  MUON_ERR_TIMEOUT = 5,      /* a bounded device-side wait expired (kernel gave up and returned) */
+  MUON_ERR_TOO_LARGE = 6     /* the matrix does not fit the fixed scratch of muon_newton_schulz_noalloc */
 } muon_status;
 
 typedef enum { MUON_F32 = 0, MUON_BF16 = 1 } muon_dtype;
@@ -119,6 +120,40 @@ MUON_API muon_status muon_newton_schulz(muon_handle_t h, const void* const* x_in
                                const int64_t* rows, const int64_t* cols, int n,
                                muon_dtype dtype, const float* coeffs, int ns_steps,
                                float eps, muon_mode mode, void* cuda_stream);
+
+/* Allocation-free Newton-Schulz of ONE matrix.  The paper has no counterpart: this
+ * entry point exists for callers that may not allocate device memory when they need
+ * the update -- runtimes that reserve all device memory for their own pool at
+ * start-up, engines that forbid allocation after initialisation, or latency-bound
+ * loops where a cudaMalloc (which can synchronise the device) is not acceptable.
+ * muon_newton_schulz allocates a workspace on first use; this function instead uses a
+ * fixed 32 MiB scratch array compiled into the library and calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *
+ * Computes what muon_newton_schulz computes in MUON_MODE_BF16 for a single matrix,
+ * with the same kernels: o_out = Newton-Schulz of x_in / (||x_in||_F + eps).
+ *  x_in, o_out   DEVICE pointers on the CURRENT device, rows x cols of `dtype`,
+ *                row-major, 16-byte aligned, not overlapping; caller-owned
+ *  status        optional DEVICE int (4-byte aligned); if not NULL, a bounded wait
+ *                that expires inside a kernel stores 1 there (the caller clears it);
+ *                if NULL, such a time-out goes unreported
+ *  coeffs, ns_steps, eps, cuda_stream   as in muon_newton_schulz
+ * Limit: the matrix must fit the scratch: with s = min(rows, cols), L = max(rows, cols)
+ * and r8(v) = v rounded up to a multiple of 8, about 4*s*r8(L) + 4*s*r8(s) bytes plus
+ * small tables must stay within 32 MiB (1024x3072 and 1536x1536 fit, 2048x2048 does
+ * not).  Larger matrices return MUON_ERR_TOO_LARGE with nothing enqueued.  Argument
+ * errors return MUON_ERR_INVALID_ARG, a device that is not compute capability 10.0
+ * MUON_ERR_UNSUPPORTED.
+ * The first call on a device, with that device current, looks up the array's device
+ * address (cudaGetSymbolAddress) and caches it; make that first call before any stream
+ * capture.  Every call uses the same array and overwrites it: calls that overlap on the
+ * GPU (other streams, other host threads) race and corrupt each other's results, and
+ * the host side is not thread-safe.  Every GPU that loads the library's kernels holds
+ * the 32 MiB until the process exits. */
+MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, void* o_out, int64_t rows,
+                                                int64_t cols, muon_dtype dtype,
+                                                const float* coeffs, int ns_steps, float eps,
+                                                int* status, void* cuda_stream);
 
 /* Waits for the handle's last enqueued work and returns its device-side status
  * (MUON_OK or MUON_ERR_TIMEOUT), clearing it. */

@@ -25,13 +25,15 @@ MUON_ERR_UNSUPPORTED = 2
 MUON_ERR_OOM = 3
 MUON_ERR_CUDA = 4
 MUON_ERR_TIMEOUT = 5
+MUON_ERR_TOO_LARGE = 6
 
 MUON_F32 = 0
 MUON_BF16 = 1
 MUON_MODE_BF16 = 0
 MUON_MODE_FP32_VALIDATE = 1
 
-EXPORTED = ("muon_init", "muon_step", "muon_newton_schulz", "muon_sync", "muon_workspace_bytes",
+EXPORTED = ("muon_init", "muon_step", "muon_newton_schulz", "muon_newton_schulz_noalloc", "muon_sync",
+            "muon_workspace_bytes",
             "muon_last_launch_count", "muon_profile_enable", "muon_profile_read", "muon_destroy",
             "muon_status_string", "muon_last_error")
 
@@ -71,6 +73,8 @@ def load_library(path: str = LIB_PATH):
     lib.muon_newton_schulz.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(i64),
                                        ctypes.POINTER(i64), i32, i32, ctypes.POINTER(f32), i32, f32, i32, vp]
     lib.muon_newton_schulz.restype = i32
+    lib.muon_newton_schulz_noalloc.argtypes = [vp, vp, i64, i64, i32, ctypes.POINTER(f32), i32, f32, vp, vp]
+    lib.muon_newton_schulz_noalloc.restype = i32
     lib.muon_sync.argtypes = [vp]
     lib.muon_sync.restype = i32
     lib.muon_workspace_bytes.argtypes = [vp]
@@ -197,6 +201,29 @@ def muon_newton_schulz(handle, xs: Sequence[torch.Tensor], outs: Sequence[torch.
     c = _coeff_array(coeffs, ns_steps)
     _check(load_library().muon_newton_schulz(handle, xin, xout, rows, cols, n, dt, c, int(ns_steps), float(eps),
                                              _mode_code(mode), _stream_ptr(stream, xs[0].device)), handle)
+
+
+def muon_newton_schulz_noalloc(x: torch.Tensor, out: torch.Tensor, coeffs=None, ns_steps: int = 5,
+                               eps: float = 1e-7, status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Allocation-free Newton-Schulz of one matrix on the current device: for callers
+    that may not allocate device memory (memory reserved up front by their own pool,
+    no allocation after start-up).  Uses a fixed 32 MiB scratch inside the library;
+    matrices that do not fit raise MuonError with code MUON_ERR_TOO_LARGE.  Calls that
+    overlap on the GPU race on that scratch.  ``status``: optional int32 CUDA tensor
+    that receives 1 if a device-side wait times out."""
+    _check_tensor(x, "x")
+    _check_tensor(out, "out")
+    if _dtype_code(x) != _dtype_code(out) or out.shape != x.shape:
+        raise ValueError("x and out must share shape and dtype")
+    st_ptr = None
+    if status is not None:
+        if not status.is_cuda or status.dtype != torch.int32:
+            raise TypeError("status must be an int32 CUDA tensor")
+        st_ptr = status.data_ptr()
+    c = _coeff_array(coeffs, ns_steps)
+    _check(load_library().muon_newton_schulz_noalloc(x.data_ptr(), out.data_ptr(), x.shape[0], x.shape[1],
+                                                     _dtype_code(x), c, int(ns_steps), float(eps), st_ptr,
+                                                     _stream_ptr(stream, x.device)))
 
 
 def muon_sync(handle) -> None:

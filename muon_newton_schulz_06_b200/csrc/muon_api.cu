@@ -759,6 +759,7 @@ const char* muon_status_string(muon_status s) {
     case MUON_ERR_OOM: return "MUON_ERR_OOM: device allocation failed";
     case MUON_ERR_CUDA: return "MUON_ERR_CUDA: CUDA call failed";
     case MUON_ERR_TIMEOUT: return "MUON_ERR_TIMEOUT: a device-side wait timed out";
+    case MUON_ERR_TOO_LARGE: return "MUON_ERR_TOO_LARGE: matrix exceeds the fixed scratch of the allocation-free entry point";
     default: return "unknown muon_status";
   }
 }
