@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", type=int, default=4, choices=[1, 2, 3, 4])
+    ap.add_argument("--layers", type=int, default=0,
+                    help="keep only the first N layers of the set (profiling captures); 0 = all")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -214,7 +216,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     cfg = args.config
-    data = synth.make_matrix_set(cfg, device=dev)
+    data = synth.make_matrix_set(cfg, device=dev, layers=list(range(args.layers)) if args.layers else None)
     W, G, M = data["W"], data["G"], data["M"]
     shapes = [(s.rows, s.cols) for s in data["specs"]]
     fl = cost.ns_flops(shapes, NS_STEPS)
@@ -340,7 +342,8 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD_TEXT[cfg], "matrices": len(shapes),
+            "config": {"workload": WORKLOAD_TEXT[cfg] + (f" (first {args.layers} layers only)" if args.layers
+                                                          else ""), "matrices": len(shapes),
                        "params": int(eb["numel"]), "ns_steps": NS_STEPS,
                        "coeffs": "quintic (3.4445, -4.7750, 2.0315) every step", "lr": LR, "momentum": MU,
                        "nesterov": True, "eps": EPS,
