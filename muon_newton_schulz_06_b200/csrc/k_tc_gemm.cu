@@ -15,34 +15,48 @@
 // triangle are computed, and the epilogue writes each upper element and its mirror.
 // Update reads X as an MN-major operand.
 //
-// CTA layout (192 threads, one CTA per SM, persistent over a cost-sorted tile list):
-//   warp 0      TMA producer (one thread): 4-stage ring of A (128 x 64) and
-//               B (256 x 64) tiles, 128-byte swizzle
-//   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.mma M=128 N=256 K=16
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns, fused scale / polynomial /
-//               update arithmetic, bf16 stores (+ mirrored stores for Gram/Poly)
-// Two 256-column accumulators in TMEM let the epilogue of tile t overlap the
-// main loop of tile t+1.  Every mbarrier wait is bounded in time; on expiry the
-// kernel writes kDevTimeout to the status word, drains its own MMAs and returns.
+// A pair of CTAs (2-CTA cluster, one CTA per SM) computes each 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = N = 256, K = 16): CTA r holds rows [128r, 128r+128) of
+// the A operand and rows / columns [128r, 128r+128) of the B operand, so each SM
+// stages only half of B and its shared memory serves 64 B/clk of operands instead of
+// 96 (the limit of the single-CTA form).  Per CTA (192 threads, persistent over the
+// cluster's share of a cost-sorted tile list):
+//   warp 0      TMA producer (one thread): 6-stage ring of 128 x 64 A and 128 x 64 B
+//               tiles, 128-byte swizzle; both CTAs' copies complete on the leader
+//               CTA's barrier (cta_group::2 form of the bulk tensor copy, no multicast)
+//   warp 1      TMEM owner; in the leader CTA also the MMA issuer (one thread), whose
+//               commits arrive on both CTAs' barriers
+//   warps 2..5  epilogue of this CTA's 128 x 256 half: tcgen05.ld 32 lanes x 32
+//               columns, fused scale / polynomial / update arithmetic, bf16 stores
+//               (+ mirrored stores for Gram/Poly)
+// Two 256-column accumulators in TMEM let the epilogue of tile t overlap the main loop
+// of tile t+1.  Every mbarrier wait is bounded in time; on expiry the kernel writes
+// kDevTimeout to the status word, tells the peer CTA, lets its own copies and MMAs
+// drain, frees TMEM and returns.
 #include "muon_internal.h"
 
 namespace muon {
 namespace {
 
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kThreadsTc = 192;
-constexpr uint32_t kABytes = kBM * kBK * 2;   // 16 KB
-constexpr uint32_t kBBytes = kBN * kBK * 2;   // 32 KB
+constexpr uint32_t kABytes = kHalf * kBK * 2;   // 16 KB: this CTA's 128 rows of A
+constexpr uint32_t kBBytes = kHalf * kBK * 2;   // 16 KB: this CTA's half of B
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr uint32_t kTmemCols = 2 * kBN;       // two fp32 accumulators of 256 columns
+constexpr uint32_t kPairTxBytes = 2 * kStageBytes;  // both CTAs' copies land on the leader's barrier
+constexpr uint32_t kTmemCols = 2 * kTile;        // two fp32 accumulators of 256 columns
 constexpr uint32_t kBarrierBytes = 256;
-constexpr uint32_t kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
+// Unused guard space after the stage ring: the MMA descriptors of the last stage never
+// address past its end, and the guard keeps any over-read inside the allocation.
+constexpr uint32_t kGuardBytes = 16384;
+constexpr uint32_t kSmemBytes = kStages * kStageBytes + kGuardBytes + kBarrierBytes + 1024;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr unsigned long long kAbortGraceNs = 1000000ull;    // 1 ms for copies in flight
 
-// tcgen05 instruction descriptor, kind::f16: D f32, A/B bf16, A K-major, N=256, M=128.
+// tcgen05 instruction descriptor, kind::f16: D f32, A/B bf16, A K-major, M = N = 256.
 __host__ __device__ constexpr uint32_t make_idesc(bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-         ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+         ((uint32_t)(kTile >> 3) << 17) | ((uint32_t)(kTile >> 4) << 24);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -76,10 +90,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -107,28 +117,72 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile 
   }
 }
 
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int x,
-                                            int y, int z) {
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(uint32_t saddr, uint32_t rank) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(saddr), "r"(rank));
+  return out;
+}
+
+__device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void remote_store_flag(uint32_t cluster_addr, int v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Bulk tensor copy into this CTA's shared memory whose completion is counted on the
+// barrier at `bar_cluster_addr` (the leader CTA's).  No multicast.
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster_addr,
+                                                 int x, int y, int z) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
+__device__ __forceinline__ void umma_pair_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
+// Arrives on the barrier at the same offset in both CTAs once this thread's MMAs finish.
+__device__ __forceinline__ void umma_commit_both(uint64_t* bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+// Arrives on this CTA's barrier once this thread's MMAs finish.
+__device__ __forceinline__ void umma_commit_local(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
+}
+
+__device__ __forceinline__ void spin_ns(unsigned long long ns) {
+  const uint64_t t0 = global_timer();
+  while (global_timer() - t0 < ns) {
+  }
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -187,7 +241,7 @@ template <int PHASE>
 __global__ void __launch_bounds__(kThreadsTc, 1) tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kGuardBytes);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
@@ -197,6 +251,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tc_kernel(const __grid_constant
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int cluster = blockIdx.x >> 1;
+  const int n_clusters = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -205,88 +262,91 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tc_kernel(const __grid_constant
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], 8);  // 4 epilogue warps in each CTA of the pair
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(kTmemCols)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers and TMEM are ready before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const uint32_t peer_abort = peer_addr(smem_u32((const void*)abort_flag), rank ^ 1u);
 
   constexpr bool kSyrk = (PHASE != kPhaseUpdate);
+  bool aborted = false;
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
+      for (int t = cluster; t < p.n_tiles && ok; t += n_clusters) {
         const TcTile tile = p.tiles[t];
         const TcGroup& g = p.g[tile.group];
         const int K = (PHASE == kPhaseGram) ? g.L : g.s;
         const int nk = (K + kBK - 1) / kBK;
         const CUtensorMap* ma = &p.map_a[tile.group];
         const CUtensorMap* mb = &p.map_b[tile.group];
-        const int row_a = tile.bi * kBM;
-        const int col_b = tile.bj * kBN;
+        const int row_a = tile.bi * kTile + (int)rank * kHalf;
+        const int col_b = tile.bj * kTile + (int)rank * kHalf;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], kStageBytes);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], kPairTxBytes);
           const uint32_t a_dst = smem_u32(smem + stage * kStageBytes);
           const uint32_t b_dst = a_dst + kABytes;
+          const uint32_t bar = peer_addr(smem_u32(&full[stage]), 0);
           const int k0 = kb * kBK;
-          tma_load_3d(a_dst, ma, &full[stage], k0, row_a, tile.mat);
+          tma_load_3d_pair(a_dst, ma, bar, k0, row_a, tile.mat);
           if (kSyrk) {
-            tma_load_3d(b_dst, ma, &full[stage], k0, col_b, tile.mat);
-            tma_load_3d(b_dst + kABytes, ma, &full[stage], k0, col_b + kBM, tile.mat);
+            tma_load_3d_pair(b_dst, ma, bar, k0, col_b, tile.mat);
           } else {
 #pragma unroll
-            for (int q = 0; q < kBN / 64; ++q)
-              tma_load_3d(b_dst + q * (64 * kBK * 2), mb, &full[stage], col_b + 64 * q, k0, tile.mat);
+            for (int q = 0; q < kHalf / 64; ++q)
+              tma_load_3d_pair(b_dst + q * (64 * kBK * 2), mb, bar, col_b + 64 * q, k0, tile.mat);
           }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok) {
+      if (!ok || *abort_flag) {
+        aborted = true;
         atomicExch(p.status, kDevTimeout);
         *abort_flag = 1;
-      }
-      // let every copy this thread armed land before the CTA can exit
-      for (int s = 0; s < kStages; ++s) {
-        // the most recent arm of stage s used parity (phase of that pass)
-        const int passes_back = (s < stage) ? 0 : 1;
-        const uint32_t par = passes_back ? (phase ^ 1u) : phase;
-        (void)mbar_wait(&full[s], par, nullptr);
+        remote_store_flag(peer_abort, 1);
+        spin_ns(kAbortGraceNs);  // copies already issued land within microseconds
+      } else if (rank == 0) {
+        // every copy armed on this barrier set has landed (all were consumed in order)
+        for (int s = 0; s < kStages; ++s) {
+          const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
+          (void)mbar_wait(&full[s], par, nullptr);
+        }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------------ MMA issuer (leader CTA)
+    if (lane == 0 && rank == 0) {
       constexpr uint32_t idesc = make_idesc(!kSyrk);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
+      for (int t = cluster; t < p.n_tiles && ok; t += n_clusters) {
         const TcTile tile = p.tiles[t];
         const TcGroup& g = p.g[tile.group];
         const int K = (PHASE == kPhaseGram) ? g.L : g.s;
         const int nk = (K + kBK - 1) / kBK;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kBN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kTile);
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
@@ -297,44 +357,47 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tc_kernel(const __grid_constant
             const uint64_t ad = sdesc(a_addr + k * 32, 16, 1024);
             const uint64_t bd = kSyrk ? sdesc(b_addr + k * 32, 16, 1024)
                                       : sdesc(b_addr + k * 2048, 64 * kBK * 2, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            umma_pair_bf16(d_tmem, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
           }
-          umma_commit(&empty[stage]);
+          umma_commit_both(&empty[stage]);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        umma_commit_both(&tfull[acc]);
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
       if (!ok) {
+        aborted = true;
         atomicExch(p.status, kDevTimeout);
         *abort_flag = 1;
+        remote_store_flag(peer_abort, 1);
       }
-      // all MMAs issued by this thread complete before TMEM is released
-      umma_commit(drain);
+      // every MMA issued by this thread completes before TMEM is released
+      umma_commit_local(drain);
       (void)mbar_wait(drain, 0, nullptr);
     }
   } else {
-    // ------------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------------ epilogue (both CTAs)
     const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    const uint32_t leader_tempty0 = peer_addr(smem_u32(&tempty[0]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x) {
+    for (int t = cluster; t < p.n_tiles; t += n_clusters) {
       const TcTile tile = p.tiles[t];
       const TcGroup& g = p.g[tile.group];
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) { ok = false; break; }
       tc_fence_after();
 
       const int s = g.s;
-      const int row0 = tile.bi * kBM + 32 * quad;  // first row of this warp
+      const int row0 = tile.bi * kTile + (int)rank * kHalf + 32 * quad;  // first row of this warp
       const int row = row0 + lane;
       const float sc = p.first_iter ? p.scale[g.gid_base + tile.mat] : 1.f;
-      const uint32_t tbase = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(acc * kBN);
+      const uint32_t tbase = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(acc * kTile);
 
       if (row0 < s) {
-        for (int c = 0; c < kBN / 32; ++c) {
-          const int col0 = tile.bj * kBN + 32 * c;
+        for (int c = 0; c < kTile / 32; ++c) {
+          const int col0 = tile.bj * kTile + 32 * c;
           if (kSyrk) {
             if (col0 >= s || col0 + 31 < row0) continue;  // outside / strictly lower block
           } else {
@@ -415,50 +478,113 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tc_kernel(const __grid_constant
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) remote_arrive(leader_tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
     if (!ok && lane == 0) {
+      aborted = true;
       atomicExch(p.status, kDevTimeout);
       *abort_flag = 1;
+      remote_store_flag(peer_abort, 1);
     }
   }
+  (void)aborted;
 
+  // Both CTAs wait here: the leader's MMAs (which write the peer's TMEM) and every copy
+  // are complete before either CTA releases TMEM or exits.
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
                  : "memory");
   }
 }
 
 template <int PHASE>
-cudaError_t launch_phase(const TcParams& p, int grid, cudaStream_t st) {
-  static uint64_t configured = 0;  // one bit per device: the attribute is set per device
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+cudaError_t set_smem_attr() {
+  return cudaFuncSetAttribute(tc_kernel<PHASE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+}
+
+struct DeviceInfo {
+  bool ready = false;
+  int clusters = 0;
+};
+DeviceInfo g_dev_info[64];
+
+// Sets the shared-memory attribute of every phase on the current device and finds how
+// many 2-CTA clusters of this kernel fit at once.
+cudaError_t device_setup(int dev) {
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  DeviceInfo& d = g_dev_info[dev];
+  if (d.ready) return cudaSuccess;
+  cudaError_t e = set_smem_attr<kPhaseGram>();
+  if (e == cudaSuccess) e = set_smem_attr<kPhasePoly>();
+  if (e == cudaSuccess) e = set_smem_attr<kPhaseUpdate>();
   if (e != cudaSuccess) return e;
-  const uint64_t bit = (dev < 64) ? (uint64_t(1) << dev) : 0;
-  if (!(configured & bit)) {
-    e = cudaFuncSetAttribute(tc_kernel<PHASE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured |= bit;
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(sms & ~1), 1, 1);
+  cfg.blockDim = dim3(kThreadsTc, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  e = cudaOccupancyMaxActiveClusters(&n, tc_kernel<kPhaseUpdate>, &cfg);
+  if (e != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = sms / 2;
   }
-  tc_kernel<PHASE><<<grid, kThreadsTc, kSmemBytes, st>>>(p);
-  return cudaGetLastError();
+  d.clusters = n;
+  d.ready = true;
+  return cudaSuccess;
+}
+
+template <int PHASE>
+cudaError_t launch_phase(const TcParams& p, int clusters, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
+  cfg.blockDim = dim3(kThreadsTc, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_kernel<PHASE>, p);
 }
 
 }  // namespace
 
-int tc_smem_bytes() { return (int)kSmemBytes; }
+int tc_grid_clusters(int n_tiles) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || device_setup(dev) != cudaSuccess) return 1;
+  int c = g_dev_info[dev].clusters;
+  if (n_tiles < c) c = n_tiles;
+  return c < 1 ? 1 : c;
+}
 
-cudaError_t launch_tc(int phase, const TcParams& p, int grid, cudaStream_t st) {
+cudaError_t launch_tc(int phase, const TcParams& p, int clusters, cudaStream_t st) {
   if (p.n_tiles == 0) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = device_setup(dev);
+  if (e != cudaSuccess) return e;
   switch (phase) {
-    case kPhaseGram: return launch_phase<kPhaseGram>(p, grid, st);
-    case kPhasePoly: return launch_phase<kPhasePoly>(p, grid, st);
-    case kPhaseUpdate: return launch_phase<kPhaseUpdate>(p, grid, st);
+    case kPhaseGram: return launch_phase<kPhaseGram>(p, clusters, st);
+    case kPhasePoly: return launch_phase<kPhasePoly>(p, clusters, st);
+    case kPhaseUpdate: return launch_phase<kPhaseUpdate>(p, clusters, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -269,15 +269,13 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
       std::vector<TcTile> syrk, upd;
       for (int gg = c.g_begin; gg < c.g_end; ++gg) {
         const GroupPlan& g = P.groups[gg];
-        const int mb = (g.s + kBM - 1) / kBM, nb_s = (g.s + kBN - 1) / kBN, nb_l = (g.L + kBN - 1) / kBN;
+        const uint16_t lg = (uint16_t)(gg - c.g_begin);
         for (int m = 0; m < g.n; ++m) {
-          for (int bi = 0; bi < mb; ++bi)
-            for (int bj = 0; bj < nb_s; ++bj)
-              if (bj * kBN + kBN - 1 >= bi * kBM)  // touches the upper triangle
-                syrk.push_back(TcTile{(uint16_t)(gg - c.g_begin), (uint16_t)m, (uint16_t)bi, (uint16_t)bj});
-          for (int bi = 0; bi < mb; ++bi)
-            for (int bj = 0; bj < nb_l; ++bj)
-              upd.push_back(TcTile{(uint16_t)(gg - c.g_begin), (uint16_t)m, (uint16_t)bi, (uint16_t)bj});
+          const size_t s0 = syrk.size(), u0 = upd.size();
+          syrk.resize(s0 + tc_syrk_tiles(g.s, lg, (uint16_t)m, nullptr));
+          tc_syrk_tiles(g.s, lg, (uint16_t)m, syrk.data() + s0);
+          upd.resize(u0 + tc_update_tiles(g.s, g.L, lg, (uint16_t)m, nullptr));
+          tc_update_tiles(g.s, g.L, lg, (uint16_t)m, upd.data() + u0);
         }
       }
       std::vector<GroupPlan> cg(P.groups.begin() + c.g_begin, P.groups.begin() + c.g_end);
@@ -333,11 +331,11 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
       const GroupPlan& g = P.groups[gg];
       muon_status s;
       for (int b = 0; b < 2; ++b) {
-        if ((s = encode_map(h, &P.map_xk[b][gg], h->ws + g.off_x[b], g.L, g.s, g.n, g.ld_x, kBK, kBM))) return s;
+        if ((s = encode_map(h, &P.map_xk[b][gg], h->ws + g.off_x[b], g.L, g.s, g.n, g.ld_x, kBK, kHalf))) return s;
         if ((s = encode_map(h, &P.map_xmn[b][gg], h->ws + g.off_x[b], g.L, g.s, g.n, g.ld_x, 64, kBK))) return s;
       }
-      if ((s = encode_map(h, &P.map_gram[gg], h->ws + g.off_gram, g.s, g.s, g.n, g.ld_s, kBK, kBM))) return s;
-      if ((s = encode_map(h, &P.map_poly[gg], h->ws + g.off_poly, g.s, g.s, g.n, g.ld_s, kBK, kBM))) return s;
+      if ((s = encode_map(h, &P.map_gram[gg], h->ws + g.off_gram, g.s, g.s, g.n, g.ld_s, kBK, kHalf))) return s;
+      if ((s = encode_map(h, &P.map_poly[gg], h->ws + g.off_poly, g.s, g.s, g.n, g.ld_s, kBK, kHalf))) return s;
     }
   }
   P.valid = true;
@@ -488,9 +486,9 @@ muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, cudaStr
         tp->cc = c[2];
         tp->scale = scale;
         tp->status = h->dev_status;
-        const int grid = std::max(1, std::min(tp->n_tiles, h->sm_count));
+        const int clusters = tc_grid_clusters(tp->n_tiles);
         prof_begin(h, st);
-        cudaError_t e = launch_tc(ph, *tp, grid, st);
+        cudaError_t e = launch_tc(ph, *tp, clusters, st);
         prof_end(h, MUON_KIND_GRAM + ph, st);
         if (e != cudaSuccess) {
           delete tp;

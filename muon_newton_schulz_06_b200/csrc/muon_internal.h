@@ -66,16 +66,19 @@ cudaError_t launch_apply(const EwParams& p, bool work_f32, int out_kind, int gri
 // Shape groups per tensor-core launch (tensor maps travel as kernel parameters).
 constexpr int kMaxGroups = 12;
 
-constexpr int kBM = 128;   // tile rows (UMMA M)
-constexpr int kBN = 256;   // tile cols (UMMA N)
-constexpr int kBK = 64;    // k-block (one 128-byte swizzle row of bf16)
+// A tile is 256 x 256 outputs computed by a pair of CTAs (a 2-CTA cluster): each CTA
+// holds 128 rows of the A operand and 128 rows (K-major) or columns (MN-major) of the
+// B operand, and accumulates its 128 x 256 half of the tile in its own TMEM.
+constexpr int kTile = 256;  // tile rows = tile cols (UMMA M = N = 256 across the pair)
+constexpr int kHalf = 128;  // rows of A / of B each CTA loads (TMA box rows)
+constexpr int kBK = 64;     // k-block (one 128-byte swizzle row of bf16)
 
 enum TcPhase : int { kPhaseGram = 0, kPhasePoly = 1, kPhaseUpdate = 2 };
 
 struct TcTile {
   uint16_t group;
   uint16_t mat;   // index inside the group
-  uint16_t bi;    // 128-row block
+  uint16_t bi;    // 256-row block
   uint16_t bj;    // 256-col block
 };
 
@@ -102,8 +105,36 @@ struct __align__(64) TcParams {
   int* status;                    // device status word
 };
 
-cudaError_t launch_tc(int phase, const TcParams& p, int grid, cudaStream_t st);
-int tc_smem_bytes();
+// Number of 2-CTA clusters to launch for n_tiles tiles on the current device.
+int tc_grid_clusters(int n_tiles);
+// Launches 2 * clusters CTAs (one cluster per tile at a time, persistent).
+cudaError_t launch_tc(int phase, const TcParams& p, int clusters, cudaStream_t st);
+
+// Tile lists of one matrix.  Symmetric products: 256 x 256 blocks (bi <= bj) of the
+// s x s result, row-block major.  Update: every 256 x 256 block of the s x L result,
+// column-block major, so that the CTAs running at one time share X's column blocks
+// and the whole polynomial matrix in L2.  Returns the count; writes when out != null.
+inline int tc_syrk_tiles(int s, uint16_t group, uint16_t mat, TcTile* out) {
+  const int nb = (s + kTile - 1) / kTile;
+  int n = 0;
+  for (int bi = 0; bi < nb; ++bi)
+    for (int bj = bi; bj < nb; ++bj) {
+      if (out) out[n] = TcTile{group, mat, (uint16_t)bi, (uint16_t)bj};
+      ++n;
+    }
+  return n;
+}
+
+inline int tc_update_tiles(int s, int L, uint16_t group, uint16_t mat, TcTile* out) {
+  const int mb = (s + kTile - 1) / kTile, nb = (L + kTile - 1) / kTile;
+  int n = 0;
+  for (int bj = 0; bj < nb; ++bj)
+    for (int bi = 0; bi < mb; ++bi) {
+      if (out) out[n] = TcTile{group, mat, (uint16_t)bi, (uint16_t)bj};
+      ++n;
+    }
+  return n;
+}
 
 // ----------------------------------------------------------------- fp32 validation path
 

@@ -85,12 +85,8 @@ extern "C" MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, voi
   const int ld_x = (L + 7) / 8 * 8, ld_s = (s + 7) / 8 * 8;
   const int tiles_c = (int)((cols + kEwTile - 1) / kEwTile);
   const int n_units = (int)((rows + kEwTile - 1) / kEwTile) * tiles_c;
-  const int mb = (s + kBM - 1) / kBM, nb_s = (s + kBN - 1) / kBN, nb_l = (L + kBN - 1) / kBN;
-  int n_syrk = 0;
-  for (int bi = 0; bi < mb; ++bi)
-    for (int bj = 0; bj < nb_s; ++bj)
-      if (bj * kBN + kBN - 1 >= bi * kBM) ++n_syrk;
-  const int n_upd = mb * nb_l;
+  const int n_syrk = tc_syrk_tiles(s, 0, 0, nullptr);
+  const int n_upd = tc_update_tiles(s, L, 0, 0, nullptr);
   if ((int64_t)n_syrk + n_upd > kMaxTiles) return MUON_ERR_TOO_LARGE;
   size_t off = 0;
   const size_t off_x0 = off; off = up(off + (size_t)s * ld_x * 2, 1024);
@@ -135,12 +131,7 @@ extern "C" MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, voi
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
 
   // ---- tile lists (Gram and Poly share the triangle list) and zeroed words
-  int t = 0;
-  for (int bi = 0; bi < mb; ++bi)
-    for (int bj = 0; bj < nb_s; ++bj)
-      if (bj * kBN + kBN - 1 >= bi * kBM) g_tiles[t++] = TcTile{0, 0, (uint16_t)bi, (uint16_t)bj};
-  for (int bi = 0; bi < mb; ++bi)
-    for (int bj = 0; bj < nb_l; ++bj) g_tiles[t++] = TcTile{0, 0, (uint16_t)bi, (uint16_t)bj};
+  const int t = tc_syrk_tiles(s, 0, 0, g_tiles) + tc_update_tiles(s, L, 0, 0, g_tiles + n_syrk);
   // pageable source: the copy is staged before the call returns, so g_tiles may be reused
   if (cudaMemcpyAsync(scr + off_tiles, g_tiles, (size_t)t * sizeof(TcTile), cudaMemcpyHostToDevice, st) !=
       cudaSuccess)
@@ -176,11 +167,11 @@ extern "C" MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, voi
   CUtensorMap xk[2], xmn[2], gram_map, poly_map;
   for (int b = 0; b < 2; ++b) {
     char* xb = scr + (b == 0 ? off_x0 : off_x1);
-    if (!encode(&xk[b], xb, L, s, ld_x, kBK, kBM) || !encode(&xmn[b], xb, L, s, ld_x, 64, kBK))
+    if (!encode(&xk[b], xb, L, s, ld_x, kBK, kHalf) || !encode(&xmn[b], xb, L, s, ld_x, 64, kBK))
       return MUON_ERR_CUDA;
   }
-  if (!encode(&gram_map, scr + off_gram, s, s, ld_s, kBK, kBM) ||
-      !encode(&poly_map, scr + off_poly, s, s, ld_s, kBK, kBM))
+  if (!encode(&gram_map, scr + off_gram, s, s, ld_s, kBK, kHalf) ||
+      !encode(&poly_map, scr + off_poly, s, s, ld_s, kBK, kHalf))
     return MUON_ERR_CUDA;
   const TcTile* dev_tiles = reinterpret_cast<const TcTile*>(scr + off_tiles);
   for (int k = 0; k < ns_steps; ++k) {
@@ -214,7 +205,7 @@ extern "C" MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, voi
       g_tc.cc = c[2];
       g_tc.scale = reinterpret_cast<const float*>(scr + off_scale);
       g_tc.status = stat;
-      if (launch_tc(ph, g_tc, std::max(1, std::min(g_tc.n_tiles, sms)), st) != cudaSuccess) return MUON_ERR_CUDA;
+      if (launch_tc(ph, g_tc, tc_grid_clusters(g_tc.n_tiles), st) != cudaSuccess) return MUON_ERR_CUDA;
     }
   }
 
