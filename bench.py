@@ -307,8 +307,8 @@ def main():
         if n == 0:
             continue
         avg_ms = kms / n
-        if kind in ("gram", "poly", "update"):
-            work = fl["per_launch"][kind]
+        if kind in ("gram", "poly", "update", "update_apply"):
+            work = fl["per_launch"]["update" if kind == "update_apply" else kind]
             ach = work / (avg_ms / 1e3) / 1e12
             kernels[kind] = {"bound": "tensor", "ms_per_launch": avg_ms, "launches": n, "achieved": ach,
                              "unit": "TFLOP/s", "work_per_launch": work,
@@ -326,7 +326,7 @@ def main():
                 "peak_kind": ("sustained bf16 (kernel timed inside a long loop), " if dk["bound"] == "tensor"
                               else "copy bandwidth, ") + pk["source"],
                 "unit": dk["unit"], "frac": dk["frac"], "traffic": None}
-    ns_ms = sum(prof[k][0] for k in ("gram", "poly", "update")) / args.steps
+    ns_ms = sum(prof[k][0] for k in ("gram", "poly", "update", "update_apply")) / args.steps
     ns_tflops = fl["algorithmic"] / (ns_ms / 1e3) / 1e12 if ns_ms > 0 else None
 
     # ---------------- CPU oracle on a bounded sample (rank 0, one GPU only)

@@ -171,8 +171,9 @@ typedef enum {
   MUON_KIND_GRAM = 1,           /* A = X X^T (scaled) */
   MUON_KIND_POLY = 2,           /* B = b A + c A^2 */
   MUON_KIND_UPDATE = 3,         /* X' = a X + B X */
-  MUON_KIND_APPLY = 4,          /* W -= lr*scale*O, or the export of O */
-  MUON_KIND_COUNT = 5
+  MUON_KIND_APPLY = 4,          /* separate W -= lr*scale*O pass, or the export of O */
+  MUON_KIND_UPDATE_APPLY = 5,   /* last update with W -= lr*scale*O fused into its epilogue */
+  MUON_KIND_COUNT = 6
 } muon_kernel_kind;
 
 /* Per-launch timing: while enabled, every launch of the handle is bracketed by two

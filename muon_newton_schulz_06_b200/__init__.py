@@ -38,7 +38,7 @@ EXPORTED = ("muon_init", "muon_step", "muon_newton_schulz", "muon_newton_schulz_
             "muon_status_string", "muon_last_error")
 
 # muon_kernel_kind
-KERNEL_KINDS = ("momentum_norm", "gram", "poly", "update", "apply")
+KERNEL_KINDS = ("momentum_norm", "gram", "poly", "update", "apply", "update_apply")
 
 
 class MuonError(RuntimeError):

@@ -10,8 +10,11 @@
 //    workspace (transposed for tall matrices); or export O into a caller buffer.
 //
 // One work unit is a 64 x 64 tile of the caller matrix; 256 threads each own 2 rows x 8
-// consecutive columns, so rows move as 16-byte vectors.  Tall matrices go through a
-// shared-memory tile to write / read the transposed workspace coalesced.
+// consecutive columns, so rows move as 16-byte vectors, and every load of a unit is
+// issued before its stores.  Tall matrices go through a shared-memory tile to write /
+// read the transposed workspace coalesced.  The norm is deterministic: each warp of a
+// unit writes one partial sum (fixed shuffle tree), and a second small kernel adds a
+// matrix's partials in a fixed order.
 #include "muon_internal.h"
 
 namespace muon {
@@ -90,28 +93,30 @@ __device__ __forceinline__ int find_mat(const EwParams& p, int unit) {
   return lo;
 }
 
-// Fixed-order block sum (deterministic for a fixed thread -> value mapping).
-__device__ __forceinline__ double block_sum(double v, double* red) {
+// Loads the 2 x 8 elements a thread owns in a 64 x 64 tile (zeros outside the matrix).
+__device__ __forceinline__ void load_tile_rows(const void* src, bool bf16, const EwMat& m, int r0, int c, int tr,
+                                               float (*v)[8]) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  double t = 0.0;
-  if (threadIdx.x == 0) {
-    for (int w = 0; w < kThreads / 32; ++w) t += red[w];
+  for (int pr = 0; pr < 2; ++pr) {
+    const int r = r0 + tr + 32 * pr;
+    const size_t base = (size_t)r * m.cols + c;
+    if (r < m.rows && c + 8 <= m.cols && m.vec_ok) {
+      ld8(src, base, bf16, v[pr]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[pr][q] = (r < m.rows && c + q < m.cols) ? ld_elem(src, base + q, bf16) : 0.f;
+    }
   }
-  return t;  // valid in thread 0
 }
 
+// Momentum + Nesterov + U (workspace) + per-warp sums of U^2.  All loads of a unit are
+// issued before any store, so each thread keeps 2 rows of G and M in flight.
 template <typename WT>
 __global__ void __launch_bounds__(kThreads)
 momentum_norm_kernel(const __grid_constant__ EwParams p) {
   __shared__ float tile[kEwTile][kEwTile + 1];
-  __shared__ double red[kThreads / 32];
-  __shared__ int is_last;
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   const int tr = tid >> 3;        // 0..31
   const int tcol = (tid & 7) * 8; // 0..56
 
@@ -121,79 +126,66 @@ momentum_norm_kernel(const __grid_constant__ EwParams p) {
     const int u = unit - m.unit_begin;
     const int r0 = (u / m.tiles_c) * kEwTile;
     const int c0 = (u % m.tiles_c) * kEwTile;
+    const int c = c0 + tcol;
     WT* work = reinterpret_cast<WT*>(m.work);
-    float ssq = 0.f;
 
+    float g[2][8], mo[2][8];
+    if (p.use_momentum) {
+      load_tile_rows(m.grad, m.grad_bf16, m, r0, c, tr, g);
+      load_tile_rows(m.mom, false, m, r0, c, tr, mo);
+    } else {
+      load_tile_rows(m.param, m.param_bf16, m, r0, c, tr, g);
+    }
+    float ssq = 0.f;
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
-      const int r = r0 + tr + 32 * pr;
-      const int c = c0 + tcol;
-      float g[8], mo[8], uu[8];
-      const bool in_row = r < m.rows;
-      const bool full = in_row && (c + 8 <= m.cols);
-      const size_t base = (size_t)r * m.cols + c;
-      if (full && m.vec_ok) {
-        if (p.use_momentum) {
-          ld8(m.grad, base, m.grad_bf16, g);
-          ld8(m.mom, base, false, mo);
-        } else {
-          ld8(m.param, base, m.param_bf16, g);
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const bool ok = in_row && (c + q < m.cols);
-          if (p.use_momentum) {
-            g[q] = ok ? ld_elem(m.grad, base + q, m.grad_bf16) : 0.f;
-            mo[q] = ok ? m.mom[base + q] : 0.f;
-          } else {
-            g[q] = ok ? ld_elem(m.param, base + q, m.param_bf16) : 0.f;
-          }
-        }
-      }
       if (p.use_momentum) {
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          const float mn = __fadd_rn(__fmul_rn(p.mu, mo[q]), g[q]);
-          mo[q] = mn;
-          uu[q] = p.nesterov ? __fadd_rn(g[q], __fmul_rn(p.mu, mn)) : mn;
+          const float mn = __fadd_rn(__fmul_rn(p.mu, mo[pr][q]), g[pr][q]);
+          mo[pr][q] = mn;
+          g[pr][q] = p.nesterov ? __fadd_rn(g[pr][q], __fmul_rn(p.mu, mn)) : mn;  // g now holds U
         }
-        if (full && m.vec_ok) {
-          st8<float>(m.mom, base, mo);
-        } else {
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            if (in_row && c + q < m.cols) m.mom[base + q] = mo[q];
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) uu[q] = g[q];
       }
 #pragma unroll
-      for (int q = 0; q < 8; ++q) ssq = fmaf(uu[q], uu[q], ssq);  // zero outside the matrix
-
-      if (!m.transposed) {
-        // workspace row r holds caller row r
-        if (full) {
-          st8<WT>(work, (size_t)r * m.ld + c, uu);
+      for (int q = 0; q < 8; ++q) ssq = fmaf(g[pr][q], g[pr][q], ssq);  // zero outside the matrix
+    }
+    if (m.transposed) __syncthreads();  // the previous unit's readers are done with `tile`
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr) {
+      const int r = r0 + tr + 32 * pr;
+      const bool in_row = r < m.rows;
+      const bool full = in_row && (c + 8 <= m.cols);
+      const size_t base = (size_t)r * m.cols + c;
+      if (p.use_momentum) {
+        if (full && m.vec_ok) {
+          st8<float>(m.mom, base, mo[pr]);
         } else {
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            if (in_row && c + q < m.cols) st1<WT>(work, (size_t)r * m.ld + c + q, uu[q]);
+            if (in_row && c + q < m.cols) m.mom[base + q] = mo[pr][q];
+        }
+      }
+      if (!m.transposed) {
+        if (full) {
+          st8<WT>(work, (size_t)r * m.ld + c, g[pr]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (in_row && c + q < m.cols) st1<WT>(work, (size_t)r * m.ld + c + q, g[pr][q]);
         }
       } else {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) tile[tr + 32 * pr][tcol + q] = uu[q];
+        for (int q = 0; q < 8; ++q) tile[tr + 32 * pr][tcol + q] = g[pr][q];
       }
     }
-
     if (m.transposed) {
       __syncthreads();
       // workspace row (c0 + j) holds caller column c0 + j, over caller rows r0..r0+63
 #pragma unroll
       for (int pr = 0; pr < 2; ++pr) {
-        const int j = tr + 32 * pr;          // caller column offset
-        const int i0 = tcol;                 // caller row offset
+        const int j = tr + 32 * pr;
+        const int i0 = tcol;
         const int wr = c0 + j;
         if (wr < m.cols) {
           float v[8];
@@ -210,26 +202,30 @@ momentum_norm_kernel(const __grid_constant__ EwParams p) {
         }
       }
     }
+    // fixed shuffle tree per warp; one partial per (unit, warp)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+    if (lane == 0) p.partials[(size_t)(m.part_base + u) * kWarpsPerUnit + warp] = ssq;
+  }
+}
 
-    const double tot = block_sum((double)ssq, red);
-    if (tid == 0) {
-      p.partials[m.part_base + u] = (float)tot;
-      __threadfence();
-      const unsigned prev = atomicAdd(&p.counters[m.gid], 1u);
-      is_last = (prev == (unsigned)(m.n_units - 1));
-    }
-    __syncthreads();
-    if (is_last) {
-      __threadfence();
-      double acc = 0.0;
-      for (int k = tid; k < m.n_units; k += kThreads) acc += (double)__ldcg(p.partials + m.part_base + k);
-      const double all = block_sum(acc, red);
-      if (tid == 0) {
-        p.scale[m.gid] = (float)(1.0 / (sqrt(all) + (double)p.eps));
-        p.counters[m.gid] = 0u;
-      }
-    }
-    __syncthreads();
+// scale[gid] = 1 / (sqrt(sum of the matrix's partials) + eps): one block per matrix,
+// fixed summation order (strided per thread, then a fixed tree), in double.
+__global__ void __launch_bounds__(kThreads)
+norm_finalize_kernel(const __grid_constant__ EwParams p) {
+  __shared__ double red[kThreads / 32];
+  const EwMat& m = p.mats[blockIdx.x];
+  const size_t b = (size_t)m.part_base * kWarpsPerUnit, n = (size_t)m.n_units * kWarpsPerUnit;
+  double acc = 0.0;
+  for (size_t k = threadIdx.x; k < n; k += kThreads) acc += (double)p.partials[b + k];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < kThreads / 32; ++w) t += red[w];
+    p.scale[m.gid] = (float)(1.0 / (sqrt(t) + (double)p.eps));
   }
 }
 
@@ -247,8 +243,11 @@ apply_kernel(const __grid_constant__ EwParams p, int out_kind) {
     const int u = unit - m.unit_begin;
     const int r0 = (u / m.tiles_c) * kEwTile;
     const int c0 = (u % m.tiles_c) * kEwTile;
+    const int c = c0 + tcol;
     const WT* work = reinterpret_cast<const WT*>(m.work);
 
+    float w[2][8], o[2][8];
+    if (out_kind == kEwApply) load_tile_rows(m.param, m.param_bf16, m, r0, c, tr, w);
     if (m.transposed) {
       __syncthreads();
       // stage workspace rows c0..c0+63 (caller columns), entries r0..r0+63 (caller rows)
@@ -256,65 +255,67 @@ apply_kernel(const __grid_constant__ EwParams p, int out_kind) {
       for (int pr = 0; pr < 2; ++pr) {
         const int j = tr + 32 * pr;
         const int wr = c0 + j;
+        float v[8];
+        const size_t wb = (size_t)wr * m.ld + r0 + tcol;
+        if (wr < m.cols && r0 + tcol + 8 <= m.rows) {
+          ld8(work, wb, sizeof(WT) == 2, v);
+        } else {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int i = r0 + tcol + q;
-          float v = 0.f;
-          if (wr < m.cols && i < m.rows) {
-            if constexpr (sizeof(WT) == 2) v = __bfloat162float(work[(size_t)wr * m.ld + i]);
-            else v = work[(size_t)wr * m.ld + i];
+          for (int q = 0; q < 8; ++q) {
+            float x = 0.f;
+            if (wr < m.cols && r0 + tcol + q < m.rows) {
+              if constexpr (sizeof(WT) == 2) x = __bfloat162float(work[wb + q]);
+              else x = work[wb + q];
+            }
+            v[q] = x;
           }
-          tile[tcol + q][j] = v;
         }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) tile[tcol + q][j] = v[q];
       }
       __syncthreads();
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) o[pr][q] = tile[tr + 32 * pr][tcol + q];
+    } else {
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) {
+        const int r = r0 + tr + 32 * pr;
+        if (r < m.rows && c + 8 <= m.cols) {
+          ld8(work, (size_t)r * m.ld + c, sizeof(WT) == 2, o[pr]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float x = 0.f;
+            if (r < m.rows && c + q < m.cols) {
+              if constexpr (sizeof(WT) == 2) x = __bfloat162float(work[(size_t)r * m.ld + c + q]);
+              else x = work[(size_t)r * m.ld + c + q];
+            }
+            o[pr][q] = x;
+          }
+        }
+      }
     }
-
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
       const int r = r0 + tr + 32 * pr;
-      const int c = c0 + tcol;
-      const bool in_row = r < m.rows;
-      if (!in_row) continue;
+      if (r >= m.rows) continue;
       const bool full = c + 8 <= m.cols;
-      float o[8];
-      if (m.transposed) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) o[q] = tile[tr + 32 * pr][tcol + q];
-      } else if (full) {
-        ld8(work, (size_t)r * m.ld + c, sizeof(WT) == 2, o);
-      } else {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float v = 0.f;
-          if (c + q < m.cols) {
-            if constexpr (sizeof(WT) == 2) v = __bfloat162float(work[(size_t)r * m.ld + c + q]);
-            else v = work[(size_t)r * m.ld + c + q];
-          }
-          o[q] = v;
-        }
-      }
       const size_t base = (size_t)r * m.cols + c;
-      float w[8];
       if (out_kind == kEwApply) {
-        if (full && m.vec_ok) {
-          ld8(m.param, base, m.param_bf16, w);
-        } else {
 #pragma unroll
-          for (int q = 0; q < 8; ++q) w[q] = (c + q < m.cols) ? ld_elem(m.param, base + q, m.param_bf16) : 0.f;
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) w[q] = __fsub_rn(w[q], __fmul_rn(m.lrs, o[q]));
+        for (int q = 0; q < 8; ++q) w[pr][q] = __fsub_rn(w[pr][q], __fmul_rn(m.lrs, o[pr][q]));
       } else {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) w[q] = o[q];
+        for (int q = 0; q < 8; ++q) w[pr][q] = o[pr][q];
       }
       if (full && m.vec_ok) {
-        st8_dyn(m.param, base, w, m.param_bf16);
+        st8_dyn(m.param, base, w[pr], m.param_bf16);
       } else {
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          if (c + q < m.cols) st1_dyn(m.param, base + q, w[q], m.param_bf16);
+          if (c + q < m.cols) st1_dyn(m.param, base + q, w[pr][q], m.param_bf16);
       }
     }
   }
@@ -326,6 +327,9 @@ cudaError_t launch_momentum_norm(const EwParams& p, bool work_f32, int grid, cud
   if (p.total_units == 0) return cudaSuccess;
   if (work_f32) momentum_norm_kernel<float><<<grid, kThreads, 0, st>>>(p);
   else momentum_norm_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  norm_finalize_kernel<<<p.n_mats, kThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 

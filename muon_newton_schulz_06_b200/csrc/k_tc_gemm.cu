@@ -237,8 +237,81 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v
   }
 }
 
-template <int PHASE>
-__global__ void __launch_bounds__(kThreadsTc, 1) tc_kernel(const __grid_constant__ TcParams p) {
+struct TcNoApply {
+  int unused;
+};
+
+// Weight update of one 32-column chunk of a fused epilogue (see TcApply).  xv holds
+// X_K in fp32; O is its bf16 rounding, as the workspace copy would hold it.  All 32
+// weight loads of the chunk are issued before any store.
+template <typename WT>
+__device__ __forceinline__ void fused_apply_chunk_t(WT* w, float lrs, bool transposed, bool vec, int s, int L,
+                                                    int row, int col0, const float* xv) {
+  float o[32], wv[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) o[j] = __bfloat162float(__float2bfloat16_rn(xv[j]));
+  if (!transposed && vec && col0 + 32 <= L) {
+    // W is s x L: this thread's 32 consecutive entries of row `row`
+    WT* p = w + (size_t)row * L + col0;
+    if constexpr (sizeof(WT) == 2) {
+      load_bf16x32(reinterpret_cast<const __nv_bfloat16*>(p), wv);
+    } else {
+      const float4* p4 = reinterpret_cast<const float4*>(p);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 v = p4[q];
+        wv[4 * q] = v.x; wv[4 * q + 1] = v.y; wv[4 * q + 2] = v.z; wv[4 * q + 3] = v.w;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) wv[j] = __fsub_rn(wv[j], __fmul_rn(lrs, o[j]));
+    if constexpr (sizeof(WT) == 2) {
+      store_bf16x32(reinterpret_cast<__nv_bfloat16*>(p), wv);
+    } else {
+      float4* p4 = reinterpret_cast<float4*>(p);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) p4[q] = make_float4(wv[4 * q], wv[4 * q + 1], wv[4 * q + 2], wv[4 * q + 3]);
+    }
+    return;
+  }
+  // element-wise: wide rows that are not 16-byte aligned or end inside the chunk, and tall
+  // matrices (W is L x s, entry (col0 + j, row); a warp covers 32 consecutive rows, so
+  // every access below is a coalesced 32-element run across the warp)
+  size_t idx[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) idx[j] = transposed ? (size_t)(col0 + j) * s + row : (size_t)row * L + col0 + j;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    float x = 0.f;
+    if (col0 + j < L) {
+      if constexpr (sizeof(WT) == 2) x = __bfloat162float(w[idx[j]]);
+      else x = w[idx[j]];
+    }
+    wv[j] = x;
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    if (col0 + j < L) {
+      const float r = __fsub_rn(wv[j], __fmul_rn(lrs, o[j]));
+      if constexpr (sizeof(WT) == 2) w[idx[j]] = __float2bfloat16_rn(r);
+      else w[idx[j]] = r;
+    }
+  }
+}
+
+__device__ __forceinline__ void fused_apply_chunk(const TcApply& ap, int s, int L, int row, int col0,
+                                                  const float* xv) {
+  const bool tr = ap.flags & kApplyTransposed, vec = ap.flags & kApplyVec;
+  if (ap.flags & kApplyBf16)
+    fused_apply_chunk_t(reinterpret_cast<__nv_bfloat16*>(ap.w), ap.lrs, tr, vec, s, L, row, col0, xv);
+  else
+    fused_apply_chunk_t(reinterpret_cast<float*>(ap.w), ap.lrs, tr, vec, s, L, row, col0, xv);
+}
+
+template <int PHASE, typename AppT>
+__global__ void __launch_bounds__(kThreadsTc, 1)
+tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) {
+  constexpr bool kFuse = sizeof(AppT) > sizeof(TcNoApply);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kGuardBytes);
@@ -428,6 +501,24 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tc_kernel(const __grid_constant
             const __nv_bfloat16* x = g.x_cur + moff;
             __nv_bfloat16* xn = g.x_next + moff;
             const float alpha = p.ca * sc;
+            if constexpr (kFuse) {
+              if (row < s) {
+                float xv[32];
+                if (col0 + 32 <= g.L) {
+                  load_bf16x32(x + (size_t)row * g.ld_x + col0, xv);
+                } else {
+#pragma unroll
+                  for (int j = 0; j < 32; ++j)
+                    xv[j] = (col0 + j < g.L) ? __bfloat162float(x[(size_t)row * g.ld_x + col0 + j]) : 0.f;
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) xv[j] = fmaf(alpha, xv[j], sc * v[j]);
+                fused_apply_chunk(reinterpret_cast<const TcApplyTable&>(app).m[g.gid_base + tile.mat -
+                                                                                reinterpret_cast<const TcApplyTable&>(app).base],
+                                  s, g.L, row, col0, xv);
+              }
+              continue;
+            }
             if (row < s) {
               float xv[32];
               if (col0 + 32 <= g.L) {
@@ -502,9 +593,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) tc_kernel(const __grid_constant
   }
 }
 
-template <int PHASE>
+template <int PHASE, typename AppT>
 cudaError_t set_smem_attr() {
-  return cudaFuncSetAttribute(tc_kernel<PHASE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  return cudaFuncSetAttribute(tc_kernel<PHASE, AppT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kSmemBytes);
 }
 
 struct DeviceInfo {
@@ -519,9 +611,10 @@ cudaError_t device_setup(int dev) {
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   DeviceInfo& d = g_dev_info[dev];
   if (d.ready) return cudaSuccess;
-  cudaError_t e = set_smem_attr<kPhaseGram>();
-  if (e == cudaSuccess) e = set_smem_attr<kPhasePoly>();
-  if (e == cudaSuccess) e = set_smem_attr<kPhaseUpdate>();
+  cudaError_t e = set_smem_attr<kPhaseGram, TcNoApply>();
+  if (e == cudaSuccess) e = set_smem_attr<kPhasePoly, TcNoApply>();
+  if (e == cudaSuccess) e = set_smem_attr<kPhaseUpdate, TcNoApply>();
+  if (e == cudaSuccess) e = set_smem_attr<kPhaseUpdate, TcApplyTable>();
   if (e != cudaSuccess) return e;
   int sms = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -538,7 +631,7 @@ cudaError_t device_setup(int dev) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  e = cudaOccupancyMaxActiveClusters(&n, tc_kernel<kPhaseUpdate>, &cfg);
+  e = cudaOccupancyMaxActiveClusters(&n, tc_kernel<kPhaseUpdate, TcNoApply>, &cfg);
   if (e != cudaSuccess || n <= 0) {
     cudaGetLastError();
     n = sms / 2;
@@ -548,8 +641,8 @@ cudaError_t device_setup(int dev) {
   return cudaSuccess;
 }
 
-template <int PHASE>
-cudaError_t launch_phase(const TcParams& p, int clusters, cudaStream_t st) {
+template <int PHASE, typename AppT>
+cudaError_t launch_phase(const TcParams& p, const AppT& app, int clusters, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
   cfg.blockDim = dim3(kThreadsTc, 1, 1);
@@ -562,7 +655,7 @@ cudaError_t launch_phase(const TcParams& p, int clusters, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tc_kernel<PHASE>, p);
+  return cudaLaunchKernelEx(&cfg, tc_kernel<PHASE, AppT>, p, app);
 }
 
 }  // namespace
@@ -581,12 +674,22 @@ cudaError_t launch_tc(int phase, const TcParams& p, int clusters, cudaStream_t s
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = device_setup(dev);
   if (e != cudaSuccess) return e;
+  const TcNoApply none{0};
   switch (phase) {
-    case kPhaseGram: return launch_phase<kPhaseGram>(p, clusters, st);
-    case kPhasePoly: return launch_phase<kPhasePoly>(p, clusters, st);
-    case kPhaseUpdate: return launch_phase<kPhaseUpdate>(p, clusters, st);
+    case kPhaseGram: return launch_phase<kPhaseGram>(p, none, clusters, st);
+    case kPhasePoly: return launch_phase<kPhasePoly>(p, none, clusters, st);
+    case kPhaseUpdate: return launch_phase<kPhaseUpdate>(p, none, clusters, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_tc_update_apply(const TcParams& p, const TcApplyTable& a, int clusters, cudaStream_t st) {
+  if (p.n_tiles == 0) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = device_setup(dev);
+  if (e != cudaSuccess) return e;
+  return launch_phase<kPhaseUpdate>(p, a, clusters, st);
 }
 
 }  // namespace muon

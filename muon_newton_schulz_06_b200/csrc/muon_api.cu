@@ -1,9 +1,11 @@
 // Host side of the Muon C ABI: argument checks, the plan (shape groups, workspace
 // layout, tile lists, TMA tensor maps) and the stream-ordered launch sequence
 //
-//   momentum_norm -> { Gram -> Poly -> Update } x ns_steps -> apply
+//   momentum_norm + norm finalize -> { Gram -> Poly -> Update } x ns_steps
 //
-// (17 launches for five steps when the shapes fit one launch per phase).  Matrices
+// where the last Update also applies W -= lr*scale*O in its epilogue (bf16 mode; in fp32
+// mode, and for the Newton-Schulz entry point, a separate apply / export pass follows).
+// 17 launches for five steps when the shapes fit one launch per phase.  Matrices
 // of equal wide-orientation shape (s, L) = (min(r,c), max(r,c)) are stacked into one
 // group, the device analogue of the per-shape-group stacking of the momentum
 // buffers that the autoresearch train.py review describes for MuonAdamW.
@@ -43,7 +45,7 @@ struct GroupPlan {
 };
 
 struct MatPlan {
-  int group = 0, idx = 0;
+  int group = 0, idx = 0, gid = 0;
   int64_t rows = 0, cols = 0;
   bool transposed = false;
   int n_units = 0, part_base = 0, tiles_c = 0;
@@ -61,9 +63,10 @@ struct Plan {
   std::vector<int64_t> sig;  // rows, cols pairs
   std::vector<GroupPlan> groups;
   std::vector<MatPlan> mats;
+  std::vector<int> mat_of_gid;  // caller index of each global (group-major) index
   std::vector<ChunkPlan> chunks;
   std::vector<TcTile> tiles;  // host copy of every chunk's tile lists
-  size_t off_partials = 0, off_counters = 0, off_scale = 0, off_tiles = 0, bytes = 0;
+  size_t off_partials = 0, off_scale = 0, off_tiles = 0, bytes = 0;
   int total_units = 0;
   // TMA maps per group (bf16 mode): X K-major (ping/pong), X MN-major (ping/pong), Gram, Poly
   std::vector<CUtensorMap> map_xk[2], map_xmn[2], map_gram, map_poly;
@@ -84,6 +87,7 @@ struct muon_handle {
   cudaEvent_t status_event = nullptr;
   bool status_pending = false;
   Plan plan;
+  TcApplyTable* apply_table = nullptr;  // host staging of the fused weight-update table
   // per-launch timing (muon_profile_enable)
   bool profiling = false;
   std::vector<cudaEvent_t> ev_free;
@@ -247,6 +251,11 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
     g.gid_base = gid;
     gid += g.n;
   }
+  P.mat_of_gid.assign(n, 0);
+  for (int i = 0; i < n; ++i) {
+    P.mats[i].gid = P.groups[P.mats[i].group].gid_base + P.mats[i].idx;
+    P.mat_of_gid[P.mats[i].gid] = i;
+  }
   // workspace layout
   size_t off = 0;
   for (auto& g : P.groups) {
@@ -257,8 +266,7 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
     g.off_gram = off; off = align_up(off + sbytes, 1024);
     g.off_poly = off; off = align_up(off + sbytes, 1024);
   }
-  P.off_partials = off; off = align_up(off + (size_t)P.total_units * 4, 256);
-  P.off_counters = off; off = align_up(off + (size_t)n * 4, 256);
+  P.off_partials = off; off = align_up(off + (size_t)P.total_units * kWarpsPerUnit * 4, 256);
   P.off_scale = off; off = align_up(off + (size_t)n * 4, 256);
   // tile lists (tensor-core path)
   if (mode == MUON_MODE_BF16) {
@@ -310,8 +318,7 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
     h->ws = static_cast<char*>(p);
     h->ws_bytes = P.bytes;
   }
-  cudaError_t e = cudaMemsetAsync(h->ws + P.off_counters, 0, (size_t)n * 4, st);
-  if (e != cudaSuccess) return cuda_fail(h, e, "counter reset");
+  cudaError_t e = cudaSuccess;
   if (!P.tiles.empty()) {
     e = cudaMemcpyAsync(h->ws + P.off_tiles, P.tiles.data(), P.tiles.size() * sizeof(TcTile),
                         cudaMemcpyHostToDevice, st);
@@ -381,7 +388,6 @@ muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, b
     ep->use_momentum = (momentum_pass && cm[b].mom != nullptr) ? 1 : 0;
     ep->eps = eps;
     ep->partials = reinterpret_cast<float*>(h->ws + P.off_partials);
-    ep->counters = reinterpret_cast<unsigned*>(h->ws + P.off_counters);
     ep->scale = reinterpret_cast<float*>(h->ws + P.off_scale);
     int units = 0;
     for (int j = 0; j < ep->n_mats; ++j) {
@@ -417,12 +423,25 @@ muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, b
     prof_end(h, momentum_pass ? MUON_KIND_MOMENTUM_NORM : MUON_KIND_APPLY, st);
     delete ep;
     if (err != cudaSuccess) return cuda_fail(h, err, momentum_pass ? "momentum/norm launch" : "apply launch");
-    h->last_launches++;
+    h->last_launches += momentum_pass ? 2 : 1;
   }
   return MUON_OK;
 }
 
-muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, cudaStream_t st) {
+// True when every chunk's matrices fit one fused weight-update table.
+bool can_fuse_apply(const Plan& P) {
+  if (P.mode != MUON_MODE_BF16) return false;
+  for (const ChunkPlan& ch : P.chunks) {
+    const GroupPlan& last = P.groups[ch.g_end - 1];
+    if (last.gid_base + last.n - P.groups[ch.g_begin].gid_base > kMaxFusedApply) return false;
+  }
+  return true;
+}
+
+// fuse_cm: caller matrices whose weight update is fused into the last Update pass
+// (nullptr: the last pass stores X_K for a separate apply / export pass).
+muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, const std::vector<CallMat>* fuse_cm,
+                      cudaStream_t st) {
   const Plan& P = h->plan;
   float* scale = reinterpret_cast<float*>(h->ws + P.off_scale);
   if (P.mode == MUON_MODE_FP32_VALIDATE) {
@@ -487,9 +506,31 @@ muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, cudaStr
         tp->scale = scale;
         tp->status = h->dev_status;
         const int clusters = tc_grid_clusters(tp->n_tiles);
-        prof_begin(h, st);
-        cudaError_t e = launch_tc(ph, *tp, clusters, st);
-        prof_end(h, MUON_KIND_GRAM + ph, st);
+        cudaError_t e = cudaSuccess;
+        if (fuse_cm && ph == kPhaseUpdate && k == ns_steps - 1) {
+          TcApplyTable& at = *h->apply_table;
+          at.base = P.groups[ch.g_begin].gid_base;
+          const GroupPlan& last = P.groups[ch.g_end - 1];
+          at.n = last.gid_base + last.n - at.base;
+          for (int j = 0; j < at.n; ++j) {
+            const int i = P.mat_of_gid[at.base + j];
+            const CallMat& c = (*fuse_cm)[i];
+            const MatPlan& m = P.mats[i];
+            TcApply& a = at.m[j];
+            a.w = c.param;
+            a.lrs = c.lrs;
+            a.flags = (uint16_t)((c.param_bf16 ? kApplyBf16 : 0) | (m.transposed ? kApplyTransposed : 0) |
+                                 (m.cols % 8 == 0 ? kApplyVec : 0));
+            a.pad = 0;
+          }
+          prof_begin(h, st);
+          e = launch_tc_update_apply(*tp, at, clusters, st);
+          prof_end(h, MUON_KIND_UPDATE_APPLY, st);
+        } else {
+          prof_begin(h, st);
+          e = launch_tc(ph, *tp, clusters, st);
+          prof_end(h, MUON_KIND_GRAM + ph, st);
+        }
         if (e != cudaSuccess) {
           delete tp;
           return cuda_fail(h, e, "tensor-core Newton-Schulz launch");
@@ -563,9 +604,14 @@ muon_status run(muon_handle* h, const std::vector<CallMat>& cm, const int64_t* r
     if ((s = build_plan(h, rows, cols, n, mode, st))) return s;
   }
   const int final_buf = ns_steps & 1;
+  const bool fuse = step && can_fuse_apply(h->plan);
+  if (fuse && !h->apply_table) {
+    h->apply_table = new (std::nothrow) TcApplyTable();
+    if (!h->apply_table) return fail(h, MUON_ERR_OOM, "host allocation of the weight-update table failed");
+  }
   if ((s = launch_elementwise(h, cm, true, 0, 0, mu, nesterov, eps, st))) return s;
-  if ((s = launch_ns(h, coeffs, ns_steps, st))) return s;
-  if ((s = launch_elementwise(h, cm, false, step ? kEwApply : kEwExport, final_buf, mu, nesterov, eps, st)))
+  if ((s = launch_ns(h, coeffs, ns_steps, fuse ? &cm : nullptr, st))) return s;
+  if (!fuse && (s = launch_elementwise(h, cm, false, step ? kEwApply : kEwExport, final_buf, mu, nesterov, eps, st)))
     return s;
   return finish_call(h, st);
 }
@@ -745,6 +791,7 @@ muon_status muon_destroy(muon_handle_t h) {
     }
     for (cudaEvent_t e : h->ev_free) cudaEventDestroy(e);
   }
+  delete h->apply_table;
   delete h;
   return s;
 }

@@ -20,8 +20,9 @@ enum DevStatus : int {
 // parameters; larger lists are split into several launches).
 constexpr int kMaxMatsPerLaunch = 192;
 
-// Square tile of one elementwise work unit.
+// Square tile of one elementwise work unit, and the norm partials it writes (one per warp).
 constexpr int kEwTile = 64;
+constexpr int kWarpsPerUnit = 8;
 
 struct EwMat {
   void* param;          // caller matrix: param (apply), or x_in (normalise-only)
@@ -33,8 +34,8 @@ struct EwMat {
   int32_t tiles_c;      // number of 64-wide tile columns of the caller matrix
   int32_t unit_begin;   // first work unit of this matrix inside the launch
   int32_t gid;          // global matrix index (partials, counters, scales)
-  int32_t part_base;    // first norm partial of this matrix
-  int32_t n_units;      // work units of this matrix (= its norm partials)
+  int32_t part_base;    // first work unit of this matrix in the partials array
+  int32_t n_units;      // work units of this matrix (kWarpsPerUnit partials each)
   uint8_t transposed;   // rows > cols: the workspace holds the transpose
   uint8_t vec_ok;       // caller rows are 16-byte aligned: vector path allowed
   uint8_t param_bf16;   // dtype of `param` (apply / export / normalise input)
@@ -50,14 +51,14 @@ struct EwParams {
   int nesterov;
   int use_momentum;     // 0: U = x_in (Newton-Schulz entry point)
   float eps;
-  float* partials;      // per-unit sum of squares
-  unsigned* counters;   // per-matrix completed units (zero between launches)
+  float* partials;      // per (unit, warp) sum of squares
   float* scale;         // per-matrix 1/(||U||_F + eps)
 };
 
 enum EwOut : int { kEwApply = 0, kEwExport = 1 };
 
 // Launchers (k_elementwise.cu).  work_f32 selects the workspace element type.
+// launch_momentum_norm enqueues two kernels: the pass and the per-matrix norm finalize.
 cudaError_t launch_momentum_norm(const EwParams& p, bool work_f32, int grid, cudaStream_t st);
 cudaError_t launch_apply(const EwParams& p, bool work_f32, int out_kind, int grid, cudaStream_t st);
 
@@ -105,10 +106,28 @@ struct __align__(64) TcParams {
   int* status;                    // device status word
 };
 
+// Weight update fused into the last Update pass: W <- RNE(fl32(W - fl32(lrs * O))) with
+// O = bf16(X_K), exactly what the separate apply pass computes; X_K itself is not stored.
+constexpr int kMaxFusedApply = 1024;
+enum : uint16_t { kApplyBf16 = 1, kApplyTransposed = 2, kApplyVec = 4 };
+struct TcApply {
+  void* w;         // caller weight, rows x cols row-major
+  float lrs;       // fl32(lr * sqrt(max(1, rows/cols)))
+  uint16_t flags;  // kApplyBf16 | kApplyTransposed (rows > cols) | kApplyVec (16-byte rows)
+  uint16_t pad;
+};
+struct __align__(16) TcApplyTable {
+  int base;        // global index of entry 0
+  int n;
+  TcApply m[kMaxFusedApply];
+};
+
 // Number of 2-CTA clusters to launch for n_tiles tiles on the current device.
 int tc_grid_clusters(int n_tiles);
 // Launches 2 * clusters CTAs (one cluster per tile at a time, persistent).
 cudaError_t launch_tc(int phase, const TcParams& p, int clusters, cudaStream_t st);
+// The last Update pass with the weight update fused into its epilogue.
+cudaError_t launch_tc_update_apply(const TcParams& p, const TcApplyTable& a, int clusters, cudaStream_t st);
 
 // Tile lists of one matrix.  Symmetric products: 256 x 256 blocks (bi <= bj) of the
 // s x s result, row-block major.  Update: every 256 x 256 block of the s x L result,

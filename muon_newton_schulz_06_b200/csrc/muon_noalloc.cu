@@ -14,8 +14,9 @@
 // device address (on the host it names a stand-in object); the first call on each
 // device, with that device current, asks the runtime for the real address with
 // cudaGetSymbolAddress and caches it.  Every call shares the array and leaves its
-// contents behind, so each call re-zeroes what must start at zero (the norm ticket
-// counter and the internal status word), and calls that overlap on the GPU race.
+// contents behind, so each call re-zeroes what must start at zero (the internal status
+// word; every other region is fully written before it is read), and calls that overlap
+// on the GPU race.
 #include <algorithm>
 #include <cmath>
 #include <cstring>
@@ -93,8 +94,7 @@ extern "C" MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, voi
   const size_t off_x1 = off; off = up(off + (size_t)s * ld_x * 2, 1024);
   const size_t off_gram = off; off = up(off + (size_t)s * ld_s * 2, 1024);
   const size_t off_poly = off; off = up(off + (size_t)s * ld_s * 2, 1024);
-  const size_t off_part = off; off = up(off + (size_t)n_units * 4, 256);
-  const size_t off_counter = off; off += 4;
+  const size_t off_part = off; off = up(off + (size_t)n_units * kWarpsPerUnit * 4, 256);
   const size_t off_scale = off; off += 4;
   const size_t off_status = off; off = up(off + 4, 256);
   const size_t off_tiles = off; off += (size_t)(n_syrk + n_upd) * sizeof(TcTile);
@@ -136,7 +136,6 @@ extern "C" MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, voi
   if (cudaMemcpyAsync(scr + off_tiles, g_tiles, (size_t)t * sizeof(TcTile), cudaMemcpyHostToDevice, st) !=
       cudaSuccess)
     return MUON_ERR_CUDA;
-  if (cudaMemsetAsync(scr + off_counter, 0, 4, st) != cudaSuccess) return MUON_ERR_CUDA;
   if (cudaMemsetAsync(scr + off_status, 0, 4, st) != cudaSuccess) return MUON_ERR_CUDA;
   int* stat = status ? status : reinterpret_cast<int*>(scr + off_status);
 
@@ -147,7 +146,6 @@ extern "C" MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, voi
   g_ew.use_momentum = 0;
   g_ew.eps = eps;
   g_ew.partials = reinterpret_cast<float*>(scr + off_part);
-  g_ew.counters = reinterpret_cast<unsigned*>(scr + off_counter);
   g_ew.scale = reinterpret_cast<float*>(scr + off_scale);
   EwMat& m = g_ew.mats[0];
   m.param = const_cast<void*>(x_in);

@@ -213,6 +213,36 @@ def test_grouped_step_matches_single_matrix_calls(mb, handle):
         assert torch.equal(a, b)
 
 
+def test_fused_and_separate_apply_agree(mb, handle):
+    """More matrices than one fused weight-update table holds (1024) take the separate
+    apply pass; the same matrices in two smaller calls take the fused epilogue.  Both
+    must give the same bits."""
+    n = 1100
+    shapes = [(16, 8) if i % 2 else (8, 24) for i in range(n)]
+    G = [synth.random_matrix(r, c, seed=2000 + i, device="cuda", dtype=torch.bfloat16) for i, (r, c) in
+         enumerate(shapes)]
+    W0 = [synth.random_matrix(r, c, seed=9000 + i, device="cuda", dtype=torch.bfloat16) for i, (r, c) in
+          enumerate(shapes)]
+    W1 = [w.clone() for w in W0]
+    M1 = [torch.zeros(r, c, device="cuda") for r, c in shapes]
+    mb.muon_step(handle, W1, G, M1, lr=0.05)
+    W2 = [w.clone() for w in W0]
+    M2 = [torch.zeros(r, c, device="cuda") for r, c in shapes]
+    h2 = mb.muon_init(0)
+    try:
+        half = n // 2
+        mb.muon_step(h2, W2[:half], G[:half], M2[:half], lr=0.05)
+        mb.muon_step(h2, W2[half:], G[half:], M2[half:], lr=0.05)
+        torch.cuda.synchronize()
+    finally:
+        mb.muon_destroy(h2)
+    torch.cuda.synchronize()
+    for a, b in zip(W1, W2):
+        assert torch.equal(a, b)
+    for a, b in zip(M1, M2):
+        assert torch.equal(a, b)
+
+
 def test_zero_gradient_leaves_weights(mb, handle):
     W = [torch.randn(256, 128, device="cuda").to(torch.bfloat16), torch.randn(64, 300, device="cuda")]
     G = [torch.zeros_like(w) for w in W]
