@@ -26,9 +26,10 @@
 //               CTA's barrier (cta_group::2 form of the bulk tensor copy, no multicast)
 //   warp 1      TMEM owner; in the leader CTA also the MMA issuer (one thread), whose
 //               commits arrive on both CTAs' barriers
-//   warps 2..5  epilogue of this CTA's 128 x 256 half: tcgen05.ld 32 lanes x 32
-//               columns, fused scale / polynomial / update arithmetic, bf16 stores
-//               (+ mirrored stores for Gram/Poly)
+//   warps 2..5  epilogue of this CTA's 128 x 256 half (one warp per TMEM lane
+//               quadrant): tcgen05.ld 32 lanes x 32 columns, fused scale / polynomial /
+//               update arithmetic; each 32 x 32 bf16 block (and, for Gram/Poly, its
+//               mirror) is staged in shared memory and written by a TMA store
 // Two 256-column accumulators in TMEM let the epilogue of tile t overlap the main loop
 // of tile t+1.  Every mbarrier wait is bounded in time; on expiry the kernel writes
 // kDevTimeout to the status word, tells the peer CTA, lets its own copies and MMAs
@@ -39,17 +40,20 @@ namespace muon {
 namespace {
 
 constexpr int kStages = 6;
-constexpr int kThreadsTc = 192;
+constexpr int kEpiWarps = 4;  // one per TMEM lane quadrant
+constexpr int kThreadsTc = 64 + 32 * kEpiWarps;
 constexpr uint32_t kABytes = kHalf * kBK * 2;   // 16 KB: this CTA's 128 rows of A
 constexpr uint32_t kBBytes = kHalf * kBK * 2;   // 16 KB: this CTA's half of B
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kPairTxBytes = 2 * kStageBytes;  // both CTAs' copies land on the leader's barrier
 constexpr uint32_t kTmemCols = 2 * kTile;        // two fp32 accumulators of 256 columns
 constexpr uint32_t kBarrierBytes = 256;
-// Unused guard space after the stage ring: the MMA descriptors of the last stage never
-// address past its end, and the guard keeps any over-read inside the allocation.
-constexpr uint32_t kGuardBytes = 16384;
-constexpr uint32_t kSmemBytes = kStages * kStageBytes + kGuardBytes + kBarrierBytes + 1024;
+// Epilogue staging for TMA stores: per epilogue warp two buffers, each a 32 x 32 bf16
+// block plus its mirror (2 KB each, 64-byte swizzle).
+constexpr uint32_t kOutBlockBytes = kOutBox * kOutBox * 2;
+constexpr uint32_t kOutWarpBytes = 2 * 2 * kOutBlockBytes;
+constexpr uint32_t kOutBytes = kEpiWarps * kOutWarpBytes;
+constexpr uint32_t kSmemBytes = kStages * kStageBytes + kOutBytes + kBarrierBytes + 1024;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr unsigned long long kAbortGraceNs = 1000000ull;    // 1 ms for copies in flight
 
@@ -179,6 +183,37 @@ __device__ __forceinline__ void umma_commit_local(uint64_t* bar) {
                : "memory");
 }
 
+// Bulk tensor store of a shared-memory block (tile mode; out-of-range parts are clipped).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// At most one committed store group may still be reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Byte offset of element (r, c) in a 32 x 32 bf16 block with 64-byte rows under the
+// 64-byte swizzle: the 16-byte chunk index is XORed with bits 1..2 of the row.
+__device__ __forceinline__ uint32_t swz64(int r, int c) {
+  return (uint32_t)(r * 64 + ((((c >> 3) ^ (r >> 1)) & 3) << 4) + (c & 7) * 2);
+}
+
+// Thread `r` writes its 32 values as row r of the block (4 x 16-byte stores).
+__device__ __forceinline__ void stage_row(uint8_t* blk, int r, const float* v) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 raw;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(v[8 * q + 2 * e], v[8 * q + 2 * e + 1]);
+    *reinterpret_cast<uint4*>(blk + r * 64 + (((q ^ (r >> 1)) & 3) << 4)) = raw;
+  }
+}
+
 __device__ __forceinline__ void spin_ns(unsigned long long ns) {
   const uint64_t t0 = global_timer();
   while (global_timer() - t0 < ns) {
@@ -277,15 +312,14 @@ __device__ __forceinline__ void fused_apply_chunk_t(WT* w, float lrs, bool trans
   // element-wise: wide rows that are not 16-byte aligned or end inside the chunk, and tall
   // matrices (W is L x s, entry (col0 + j, row); a warp covers 32 consecutive rows, so
   // every access below is a coalesced 32-element run across the warp)
-  size_t idx[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) idx[j] = transposed ? (size_t)(col0 + j) * s + row : (size_t)row * L + col0 + j;
+  WT* p0 = transposed ? w + (size_t)col0 * s + row : w + (size_t)row * L + col0;
+  const size_t stride = transposed ? (size_t)s : 1;
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
     float x = 0.f;
     if (col0 + j < L) {
-      if constexpr (sizeof(WT) == 2) x = __bfloat162float(w[idx[j]]);
-      else x = w[idx[j]];
+      if constexpr (sizeof(WT) == 2) x = __bfloat162float(p0[j * stride]);
+      else x = p0[j * stride];
     }
     wv[j] = x;
   }
@@ -293,8 +327,8 @@ __device__ __forceinline__ void fused_apply_chunk_t(WT* w, float lrs, bool trans
   for (int j = 0; j < 32; ++j) {
     if (col0 + j < L) {
       const float r = __fsub_rn(wv[j], __fmul_rn(lrs, o[j]));
-      if constexpr (sizeof(WT) == 2) w[idx[j]] = __float2bfloat16_rn(r);
-      else w[idx[j]] = r;
+      if constexpr (sizeof(WT) == 2) p0[j * stride] = __float2bfloat16_rn(r);
+      else p0[j * stride] = r;
     }
   }
 }
@@ -314,7 +348,8 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
   constexpr bool kFuse = sizeof(AppT) > sizeof(TcNoApply);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kGuardBytes);
+  uint8_t* out_stage = smem + kStages * kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kOutBytes);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
@@ -335,7 +370,7 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 8);  // 4 epilogue warps in each CTA of the pair
+      mbar_init(&tempty[a], 2 * kEpiWarps);  // every epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -451,7 +486,10 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
     }
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
-    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    const int quad = warp & 3;                       // TMEM lane quadrant this warp may access
+    uint8_t* my_stage = out_stage + (warp - 2) * kOutWarpBytes;
+    uint32_t n_out = 0;                              // staged blocks so far (buffer parity)
+    const int c_begin = ((warp - 2) / 4) * (kTile / 32 * 4 / kEpiWarps);  // first 32-column chunk
     const uint32_t leader_tempty0 = peer_addr(smem_u32(&tempty[0]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -469,7 +507,7 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
       const uint32_t tbase = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(acc * kTile);
 
       if (row0 < s) {
-        for (int c = 0; c < kTile / 32; ++c) {
+        for (int c = c_begin; c < c_begin + kTile / 32 * 4 / kEpiWarps; ++c) {
           const int col0 = tile.bj * kTile + 32 * c;
           if (kSyrk) {
             if (col0 >= s || col0 + 31 < row0) continue;  // outside / strictly lower block
@@ -519,52 +557,61 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
               }
               continue;
             }
-            if (row < s) {
-              float xv[32];
-              if (col0 + 32 <= g.L) {
-                load_bf16x32(x + (size_t)row * g.ld_x + col0, xv);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) xv[j] = fmaf(alpha, xv[j], sc * v[j]);
-                store_bf16x32(xn + (size_t)row * g.ld_x + col0, xv);
-              } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                  if (col0 + j < g.L) {
-                    const size_t o = (size_t)row * g.ld_x + col0 + j;
-                    xn[o] = __float2bfloat16_rn(fmaf(alpha, __bfloat162float(x[o]), sc * v[j]));
-                  }
-                }
-              }
-            }
-            continue;
-          }
-          // symmetric store: upper element (row, col) and its mirror (col, row)
-          __nv_bfloat16* out = (PHASE == kPhaseGram ? g.gram : g.poly) + (size_t)tile.mat * s * g.ld_s;
-          if (row < s) {
-            if (col0 >= row0 + 32) {
-              if (col0 + 32 <= s) {
-                store_bf16x32(out + (size_t)row * g.ld_s + col0, v);
-              } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  if (col0 + j < s) out[(size_t)row * g.ld_s + col0 + j] = __float2bfloat16_rn(v[j]);
-              }
+            (void)xn;
+            float xv[32];
+            if (row < s && col0 + 32 <= g.L) {
+              load_bf16x32(x + (size_t)row * g.ld_x + col0, xv);
+            } else {
 #pragma unroll
               for (int j = 0; j < 32; ++j)
-                if (col0 + j < s) out[(size_t)(col0 + j) * g.ld_s + row] = __float2bfloat16_rn(v[j]);
-            } else {
-              // diagonal 32 x 32 block (col0 == row0)
+                xv[j] = (row < s && col0 + j < g.L) ? __bfloat162float(x[(size_t)row * g.ld_x + col0 + j]) : 0.f;
+            }
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int col = col0 + j;
-                if (col < s && col >= row) {
-                  const __nv_bfloat16 b = __float2bfloat16_rn(v[j]);
-                  out[(size_t)row * g.ld_s + col] = b;
-                  if (col > row) out[(size_t)col * g.ld_s + row] = b;
-                }
+            for (int j = 0; j < 32; ++j) xv[j] = fmaf(alpha, xv[j], sc * v[j]);
+            uint8_t* blk = my_stage + (n_out & 1) * 2 * kOutBlockBytes;
+            if (lane == 0) bulk_wait_read_1();
+            __syncwarp();
+            stage_row(blk, lane, xv);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&p.map_out[tile.group], smem_u32(blk), col0, row0, tile.mat);
+              bulk_commit();
+            }
+            ++n_out;
+            continue;
+          }
+          // symmetric store: the block (row0.., col0..) and its mirror (col0.., row0..),
+          // both built from the upper-triangle values so the result is exactly symmetric
+          uint8_t* blk = my_stage + (n_out & 1) * 2 * kOutBlockBytes;
+          if (lane == 0) bulk_wait_read_1();
+          __syncwarp();
+          const bool upper = col0 >= row0 + 32;
+          if (upper) {
+            stage_row(blk, lane, v);
+            uint8_t* mir = blk + kOutBlockBytes;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              *reinterpret_cast<__nv_bfloat16*>(mir + swz64(j, lane)) = __float2bfloat16_rn(v[j]);
+          } else {
+            // diagonal block (col0 == row0): element (lane, j) for j >= lane, mirrored below
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j >= lane) {
+                const __nv_bfloat16 b = __float2bfloat16_rn(v[j]);
+                *reinterpret_cast<__nv_bfloat16*>(blk + swz64(lane, j)) = b;
+                if (j > lane) *reinterpret_cast<__nv_bfloat16*>(blk + swz64(j, lane)) = b;
               }
             }
           }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&p.map_out[tile.group], smem_u32(blk), col0, row0, tile.mat);
+            if (upper) tma_store_3d(&p.map_out[tile.group], smem_u32(blk + kOutBlockBytes), row0, col0, tile.mat);
+            bulk_commit();
+          }
+          ++n_out;
         }
       }
       tc_fence_before();
@@ -572,6 +619,7 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
       if (lane == 0) remote_arrive(leader_tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (lane == 0) bulk_wait_all();  // this warp's stores are complete and its staging is free
     if (!ok && lane == 0) {
       aborted = true;
       atomicExch(p.status, kDevTimeout);

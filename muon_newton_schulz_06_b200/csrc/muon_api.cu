@@ -17,7 +17,7 @@
 #include <string>
 #include <vector>
 
-#include "../../include/muon.h"
+#include "muon.h"
 #include "muon_internal.h"
 
 using namespace muon;
@@ -70,6 +70,8 @@ struct Plan {
   int total_units = 0;
   // TMA maps per group (bf16 mode): X K-major (ping/pong), X MN-major (ping/pong), Gram, Poly
   std::vector<CUtensorMap> map_xk[2], map_xmn[2], map_gram, map_poly;
+  // output maps (32 x 32 boxes, 64-byte swizzle) for the epilogue's TMA stores
+  std::vector<CUtensorMap> map_xout[2], map_gram_out, map_poly_out;
 };
 
 }  // namespace
@@ -197,13 +199,14 @@ void sort_tiles(std::vector<TcTile>& t, const std::vector<GroupPlan>& groups, in
 }
 
 muon_status encode_map(muon_handle* h, CUtensorMap* map, void* base, int inner, int rows, int n, int ld,
-                       int box_inner, int box_rows) {
+                       int box_inner, int box_rows,
+                       CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)n};
   cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)ld * 2 * (cuuint64_t)rows};
   cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = h->encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(h, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return MUON_OK;
@@ -331,18 +334,30 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
     for (int b = 0; b < 2; ++b) {
       P.map_xk[b].resize(ng);
       P.map_xmn[b].resize(ng);
+      P.map_xout[b].resize(ng);
     }
     P.map_gram.resize(ng);
     P.map_poly.resize(ng);
+    P.map_gram_out.resize(ng);
+    P.map_poly_out.resize(ng);
     for (size_t gg = 0; gg < ng; ++gg) {
       const GroupPlan& g = P.groups[gg];
       muon_status s;
       for (int b = 0; b < 2; ++b) {
         if ((s = encode_map(h, &P.map_xk[b][gg], h->ws + g.off_x[b], g.L, g.s, g.n, g.ld_x, kBK, kHalf))) return s;
         if ((s = encode_map(h, &P.map_xmn[b][gg], h->ws + g.off_x[b], g.L, g.s, g.n, g.ld_x, 64, kBK))) return s;
+        if ((s = encode_map(h, &P.map_xout[b][gg], h->ws + g.off_x[b], g.L, g.s, g.n, g.ld_x, kOutBox, kOutBox,
+                            CU_TENSOR_MAP_SWIZZLE_64B)))
+          return s;
       }
       if ((s = encode_map(h, &P.map_gram[gg], h->ws + g.off_gram, g.s, g.s, g.n, g.ld_s, kBK, kHalf))) return s;
       if ((s = encode_map(h, &P.map_poly[gg], h->ws + g.off_poly, g.s, g.s, g.n, g.ld_s, kBK, kHalf))) return s;
+      if ((s = encode_map(h, &P.map_gram_out[gg], h->ws + g.off_gram, g.s, g.s, g.n, g.ld_s, kOutBox, kOutBox,
+                          CU_TENSOR_MAP_SWIZZLE_64B)))
+        return s;
+      if ((s = encode_map(h, &P.map_poly_out[gg], h->ws + g.off_poly, g.s, g.s, g.n, g.ld_s, kOutBox, kOutBox,
+                          CU_TENSOR_MAP_SWIZZLE_64B)))
+        return s;
     }
   }
   P.valid = true;
@@ -490,11 +505,14 @@ muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, const s
           t.poly = reinterpret_cast<__nv_bfloat16*>(h->ws + g.off_poly);
           if (ph == kPhaseGram) {
             tp->map_a[li] = P.map_xk[cur][gg];
+            tp->map_out[li] = P.map_gram_out[gg];
           } else if (ph == kPhasePoly) {
             tp->map_a[li] = P.map_gram[gg];
+            tp->map_out[li] = P.map_poly_out[gg];
           } else {
             tp->map_a[li] = P.map_poly[gg];
             tp->map_b[li] = P.map_xmn[cur][gg];
+            tp->map_out[li] = P.map_xout[cur ^ 1][gg];
           }
         }
         tp->tiles = reinterpret_cast<const TcTile*>(h->ws + P.off_tiles) + ch.off_tiles[ph];

@@ -94,9 +94,14 @@ struct TcGroup {
   __nv_bfloat16* poly;   // [n][s][ld_s]
 };
 
+// Output blocks are written by TMA bulk-tensor stores of 32 x 32 bf16 blocks staged in
+// shared memory with the 64-byte swizzle.
+constexpr int kOutBox = 32;
+
 struct __align__(64) TcParams {
-  CUtensorMap map_a[kMaxGroups];  // A operand (K-major, box 64 x 128)
-  CUtensorMap map_b[kMaxGroups];  // B operand (K-major box 64 x 128, or MN-major box 64 x 64)
+  CUtensorMap map_a[kMaxGroups];    // A operand (K-major, box 64 x 128)
+  CUtensorMap map_b[kMaxGroups];    // B operand (K-major box 64 x 128, or MN-major box 64 x 64)
+  CUtensorMap map_out[kMaxGroups];  // output (X_next / Gram / Poly), box 32 x 32, 64-byte swizzle
   TcGroup g[kMaxGroups];
   const TcTile* tiles;
   int n_tiles;

@@ -21,7 +21,7 @@
 #include <cmath>
 #include <cstring>
 
-#include "../../include/muon.h"
+#include "muon.h"
 #include "muon_internal.h"
 
 using namespace muon;
@@ -49,13 +49,14 @@ TcParams g_tc;
 
 size_t up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-bool encode(CUtensorMap* map, void* base, int inner, int rows, int ld, int box_inner, int box_rows) {
+bool encode(CUtensorMap* map, void* base, int inner, int rows, int ld, int box_inner, int box_rows,
+            CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, 1};
   cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)ld * 2 * (cuuint64_t)rows};
   cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -162,14 +163,17 @@ extern "C" MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, voi
   if (launch_momentum_norm(g_ew, false, ew_grid, st) != cudaSuccess) return MUON_ERR_CUDA;
 
   // ---- Newton-Schulz steps on the tensor cores
-  CUtensorMap xk[2], xmn[2], gram_map, poly_map;
+  CUtensorMap xk[2], xmn[2], xout[2], gram_map, poly_map, gram_out, poly_out;
   for (int b = 0; b < 2; ++b) {
     char* xb = scr + (b == 0 ? off_x0 : off_x1);
-    if (!encode(&xk[b], xb, L, s, ld_x, kBK, kHalf) || !encode(&xmn[b], xb, L, s, ld_x, 64, kBK))
+    if (!encode(&xk[b], xb, L, s, ld_x, kBK, kHalf) || !encode(&xmn[b], xb, L, s, ld_x, 64, kBK) ||
+        !encode(&xout[b], xb, L, s, ld_x, kOutBox, kOutBox, CU_TENSOR_MAP_SWIZZLE_64B))
       return MUON_ERR_CUDA;
   }
   if (!encode(&gram_map, scr + off_gram, s, s, ld_s, kBK, kHalf) ||
-      !encode(&poly_map, scr + off_poly, s, s, ld_s, kBK, kHalf))
+      !encode(&poly_map, scr + off_poly, s, s, ld_s, kBK, kHalf) ||
+      !encode(&gram_out, scr + off_gram, s, s, ld_s, kOutBox, kOutBox, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !encode(&poly_out, scr + off_poly, s, s, ld_s, kOutBox, kOutBox, CU_TENSOR_MAP_SWIZZLE_64B))
     return MUON_ERR_CUDA;
   const TcTile* dev_tiles = reinterpret_cast<const TcTile*>(scr + off_tiles);
   for (int k = 0; k < ns_steps; ++k) {
@@ -189,11 +193,14 @@ extern "C" MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, voi
       g.poly = reinterpret_cast<__nv_bfloat16*>(scr + off_poly);
       if (ph == kPhaseGram) {
         g_tc.map_a[0] = xk[cur];
+        g_tc.map_out[0] = gram_out;
       } else if (ph == kPhasePoly) {
         g_tc.map_a[0] = gram_map;
+        g_tc.map_out[0] = poly_out;
       } else {
         g_tc.map_a[0] = poly_map;
         g_tc.map_b[0] = xmn[cur];
+        g_tc.map_out[0] = xout[cur ^ 1];
       }
       g_tc.tiles = ph == kPhaseUpdate ? dev_tiles + n_syrk : dev_tiles;
       g_tc.n_tiles = ph == kPhaseUpdate ? n_upd : n_syrk;
