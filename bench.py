@@ -154,7 +154,7 @@ def oracle_sample(config, seconds, device_data=None):
 
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
+    rank, _, _ = dist_env()
     if rank != 0:
         return
     import synth
@@ -192,6 +192,30 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ multi-rank plumbing
+
+def dist_env():
+    """(rank, world, local_rank) from the torchrun environment (1 process if absent)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time: every rank passes its own device time, all get the max."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], device=device, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(work_per_step, steps, world, ms_max):
+    """Whole-job rate of `world` replicas that each did `steps` steps of `work_per_step`
+    (weak scaling), timed by the slowest rank; in work units per second / 1e12."""
+    return work_per_step * steps * world / (ms_max / 1e3) / 1e12
+
+
 # ------------------------------------------------------------------ our arm
 
 def main():
@@ -206,9 +230,7 @@ def main():
     import synth
     from muon_newton_schulz_06_b200 import cost
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -266,11 +288,8 @@ def main():
     ms = e0.elapsed_time(e1)
     prof = mb.muon_profile_read(h)
     mb.muon_profile_enable(h, False)
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
-    value = fl["algorithmic"] * args.steps * world / (ms_max / 1e3) / 1e12
+    ms_max = max_over_ranks(ms, world, dev)
+    value = replica_throughput(fl["algorithmic"], args.steps, world, ms_max)
 
     # ---------------- end to end: pinned host gradients in, updated weights out, every step
     e2e = None
@@ -292,11 +311,8 @@ def main():
                 wh.copy_(wd, non_blocking=True)
         e3.record(stream)
         torch.cuda.synchronize()
-        t2 = torch.tensor([e2.elapsed_time(e3)], device=dev, dtype=torch.float64)
-        if world > 1:
-            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t2.item())
-        e2e = {"value": fl["algorithmic"] * args.steps * world / (ms_e2e / 1e3) / 1e12, "unit": UNIT,
+        ms_e2e = max_over_ranks(e2.elapsed_time(e3), world, dev)
+        e2e = {"value": replica_throughput(fl["algorithmic"], args.steps, world, ms_e2e), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / args.steps}
         del g_host, w_host
 

@@ -159,6 +159,14 @@ MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, void* o_out, i
  * (MUON_OK or MUON_ERR_TIMEOUT), clearing it. */
 MUON_API muon_status muon_sync(muon_handle_t h);
 
+/* Diagnostic for the time-out path: enqueues on `cuda_stream` one kernel thread that
+ * waits, with the library's bounded wait, on a barrier that nothing ever completes.
+ * After limit_ns nanoseconds (0 .. 10e9) it gives up and records a time-out in the
+ * handle's device status, which muon_sync or the next call then returns as
+ * MUON_ERR_TIMEOUT (and clears).  The GPU context stays usable.  Returns
+ * MUON_ERR_INVALID_ARG for a NULL handle or a limit out of range. */
+MUON_API muon_status muon_selftest_wait_timeout(muon_handle_t h, int64_t limit_ns, void* cuda_stream);
+
 /* Bytes of device workspace the handle currently holds. */
 MUON_API int64_t muon_workspace_bytes(muon_handle_t h);
 

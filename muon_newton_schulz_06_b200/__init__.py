@@ -33,7 +33,7 @@ MUON_MODE_BF16 = 0
 MUON_MODE_FP32_VALIDATE = 1
 
 EXPORTED = ("muon_init", "muon_step", "muon_newton_schulz", "muon_newton_schulz_noalloc", "muon_sync",
-            "muon_workspace_bytes",
+            "muon_selftest_wait_timeout", "muon_workspace_bytes",
             "muon_last_launch_count", "muon_profile_enable", "muon_profile_read", "muon_destroy",
             "muon_status_string", "muon_last_error")
 
@@ -75,6 +75,8 @@ def load_library(path: str = LIB_PATH):
     lib.muon_newton_schulz.restype = i32
     lib.muon_newton_schulz_noalloc.argtypes = [vp, vp, i64, i64, i32, ctypes.POINTER(f32), i32, f32, vp, vp]
     lib.muon_newton_schulz_noalloc.restype = i32
+    lib.muon_selftest_wait_timeout.argtypes = [vp, i64, vp]
+    lib.muon_selftest_wait_timeout.restype = i32
     lib.muon_sync.argtypes = [vp]
     lib.muon_sync.restype = i32
     lib.muon_workspace_bytes.argtypes = [vp]
@@ -224,6 +226,12 @@ def muon_newton_schulz_noalloc(x: torch.Tensor, out: torch.Tensor, coeffs=None, 
     _check(load_library().muon_newton_schulz_noalloc(x.data_ptr(), out.data_ptr(), x.shape[0], x.shape[1],
                                                      _dtype_code(x), c, int(ns_steps), float(eps), st_ptr,
                                                      _stream_ptr(stream, x.device)))
+
+
+def muon_selftest_wait_timeout(handle, limit_ns: int, stream=None) -> None:
+    """Enqueues the bounded-wait diagnostic (see include/muon.h); the next muon_sync
+    raises MuonError with code MUON_ERR_TIMEOUT."""
+    _check(load_library().muon_selftest_wait_timeout(handle, int(limit_ns), _stream_ptr(stream, None)), handle)
 
 
 def muon_sync(handle) -> None:

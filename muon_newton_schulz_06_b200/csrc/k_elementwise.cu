@@ -10,8 +10,8 @@
 //    workspace (transposed for tall matrices); or export O into a caller buffer.
 //
 // One work unit is a 64 x 64 tile of the caller matrix; 256 threads each own 2 rows x 8
-// consecutive columns, so rows move as 16-byte vectors, and every load of a unit is
-// issued before its stores.  Tall matrices go through a shared-memory tile to write /
+// consecutive columns, so rows move as 16-byte vectors (streaming cache hints: every
+// byte is touched once per pass), and every load of a unit is issued before its stores.  Tall matrices go through a shared-memory tile to write /
 // read the transposed workspace coalesced.  The norm is deterministic: each warp of a
 // unit writes one partial sum (fixed shuffle tree), and a second small kernel adds a
 // matrix's partials in a fixed order.
@@ -29,7 +29,7 @@ __device__ __forceinline__ float ld_elem(const void* p, size_t i, bool bf16) {
 
 __device__ __forceinline__ void ld8(const void* p, size_t i, bool bf16, float* v) {
   if (bf16) {
-    uint4 raw = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p) + i);
+    uint4 raw = __ldcs(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p) + i));
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -39,7 +39,7 @@ __device__ __forceinline__ void ld8(const void* p, size_t i, bool bf16, float* v
     }
   } else {
     const float4* f = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p) + i);
-    float4 a = f[0], b = f[1];
+    float4 a = __ldcs(f), b = __ldcs(f + 1);
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   }
@@ -51,8 +51,8 @@ __device__ __forceinline__ void st8(T* p, size_t i, const float* v);
 template <>
 __device__ __forceinline__ void st8<float>(float* p, size_t i, const float* v) {
   float4* f = reinterpret_cast<float4*>(p + i);
-  f[0] = make_float4(v[0], v[1], v[2], v[3]);
-  f[1] = make_float4(v[4], v[5], v[6], v[7]);
+  __stcs(f, make_float4(v[0], v[1], v[2], v[3]));
+  __stcs(f + 1, make_float4(v[4], v[5], v[6], v[7]));
 }
 
 template <>

@@ -106,9 +106,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: false on time-out, or (when abort_flag is given) once another role of
+// Bounded wait: false after limit_ns, or (when abort_flag is given) once another role of
 // the CTA gave up.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                       unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer();
   uint32_t n = 0;
@@ -116,8 +117,19 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile 
     if (mbar_try_wait(bar, parity)) return true;
     if ((++n & 63u) == 0) {
       if (abort_flag != nullptr && *abort_flag) return false;
-      if (global_timer() - t0 > kWaitLimitNs) return false;
+      if (global_timer() - t0 > limit_ns) return false;
     }
+  }
+}
+
+// Diagnostic: one thread waits, with the same bounded wait as the engine, on a barrier
+// that nothing ever completes, and records the time-out in the status word.
+__global__ void wait_selftest_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (!mbar_wait(&bar, 0, nullptr, limit_ns)) atomicExch(status, kDevTimeout);
   }
 }
 
@@ -729,6 +741,11 @@ cudaError_t launch_tc(int phase, const TcParams& p, int clusters, cudaStream_t s
     case kPhaseUpdate: return launch_phase<kPhaseUpdate>(p, none, clusters, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_wait_selftest(int* status, unsigned long long limit_ns, cudaStream_t st) {
+  wait_selftest_kernel<<<1, 32, 0, st>>>(status, limit_ns);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_tc_update_apply(const TcParams& p, const TcApplyTable& a, int clusters, cudaStream_t st) {

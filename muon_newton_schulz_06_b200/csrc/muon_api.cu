@@ -750,6 +750,22 @@ muon_status muon_newton_schulz(muon_handle_t h, const void* const* x_in, void* c
   return run(h, cm, rows, cols, false, 0.f, 0, coeffs, ns_steps, eps, mode, static_cast<cudaStream_t>(cuda_stream));
 }
 
+muon_status muon_selftest_wait_timeout(muon_handle_t h, int64_t limit_ns, void* cuda_stream) {
+  if (!h) return MUON_ERR_INVALID_ARG;
+  h->err.clear();
+  if (limit_ns < 0 || limit_ns > 10000000000ll) return fail(h, MUON_ERR_INVALID_ARG, "limit_ns out of range");
+  DeviceGuard dg(h->device);
+  if (!dg.ok) return fail(h, MUON_ERR_CUDA, "cannot select device %d", h->device);
+  muon_status s = ensure_status(h);
+  if (s) return s;
+  if ((s = poll_status(h, false))) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e = launch_wait_selftest(h->dev_status, (unsigned long long)limit_ns, st);
+  if (e != cudaSuccess) return cuda_fail(h, e, "self-test launch");
+  h->last_launches = 1;
+  return finish_call(h, st);
+}
+
 muon_status muon_sync(muon_handle_t h) {
   if (!h) return MUON_ERR_INVALID_ARG;
   DeviceGuard dg(h->device);

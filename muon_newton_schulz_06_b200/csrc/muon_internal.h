@@ -131,6 +131,8 @@ struct __align__(16) TcApplyTable {
 int tc_grid_clusters(int n_tiles);
 // Launches 2 * clusters CTAs (one cluster per tile at a time, persistent).
 cudaError_t launch_tc(int phase, const TcParams& p, int clusters, cudaStream_t st);
+// Diagnostic kernel: a bounded wait on a barrier that nothing completes (k_tc_gemm.cu).
+cudaError_t launch_wait_selftest(int* status, unsigned long long limit_ns, cudaStream_t st);
 // The last Update pass with the weight update fused into its epilogue.
 cudaError_t launch_tc_update_apply(const TcParams& p, const TcApplyTable& a, int clusters, cudaStream_t st);
 
