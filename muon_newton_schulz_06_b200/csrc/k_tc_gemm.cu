@@ -39,7 +39,8 @@
 namespace muon {
 namespace {
 
-constexpr int kStages = 6;
+// Stage ring depth per phase (Poly keeps one stage less to fit its larger staging area).
+__host__ __device__ constexpr int stages_for(int phase) { return phase == 1 ? 5 : 6; }
 constexpr int kEpiWarps = 4;  // one per TMEM lane quadrant
 constexpr int kThreadsTc = 64 + 32 * kEpiWarps;
 constexpr uint32_t kABytes = kHalf * kBK * 2;   // 16 KB: this CTA's 128 rows of A
@@ -48,12 +49,18 @@ constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kPairTxBytes = 2 * kStageBytes;  // both CTAs' copies land on the leader's barrier
 constexpr uint32_t kTmemCols = 2 * kTile;        // two fp32 accumulators of 256 columns
 constexpr uint32_t kBarrierBytes = 256;
-// Epilogue staging for TMA stores: per epilogue warp two buffers, each a 32 x 32 bf16
-// block plus its mirror (2 KB each, 64-byte swizzle).
+// Epilogue staging per warp (32 x 32 bf16 blocks of 2 KB, 64-byte swizzle), double
+// buffered: output blocks for the TMA stores (Gram/Poly: block + mirror; Update: block)
+// and, for Poly and Update, the prefetched input block (A, or X) of the next chunk.
 constexpr uint32_t kOutBlockBytes = kOutBox * kOutBox * 2;
-constexpr uint32_t kOutWarpBytes = 2 * 2 * kOutBlockBytes;
-constexpr uint32_t kOutBytes = kEpiWarps * kOutWarpBytes;
-constexpr uint32_t kSmemBytes = kStages * kStageBytes + kOutBytes + kBarrierBytes + 1024;
+__host__ __device__ constexpr uint32_t out_bytes_for(int phase) { return 2u * (phase == 2 ? 1u : 2u) * kOutBlockBytes; }
+__host__ __device__ constexpr uint32_t in_bytes_for(int phase) { return phase == 0 ? 0u : 2u * kOutBlockBytes; }
+__host__ __device__ constexpr uint32_t warp_stage_bytes_for(int phase) { return out_bytes_for(phase) + in_bytes_for(phase); }
+__host__ __device__ constexpr uint32_t smem_bytes_for(int phase) {
+  return (uint32_t)stages_for(phase) * kStageBytes + kEpiWarps * warp_stage_bytes_for(phase) + kBarrierBytes + 1024;
+}
+static_assert(smem_bytes_for(0) <= 232448 && smem_bytes_for(1) <= 232448 && smem_bytes_for(2) <= 232448,
+              "shared memory per CTA");
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr unsigned long long kAbortGraceNs = 1000000ull;    // 1 ms for copies in flight
 
@@ -193,6 +200,31 @@ __device__ __forceinline__ void umma_commit_both(uint64_t* bar) {
 __device__ __forceinline__ void umma_commit_local(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
+}
+
+// Bulk tensor copy into this CTA's shared memory, completing on this CTA's barrier.
+__device__ __forceinline__ void tma_load_3d_local(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                                  int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// Thread `r` reads row r of a staged 32 x 32 bf16 block (4 x 16-byte loads).
+__device__ __forceinline__ void unstage_row(const uint8_t* blk, int r, float* v) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(blk + r * 64 + (((q ^ (r >> 1)) & 3) << 4));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h[e]);
+      v[8 * q + 2 * e] = f.x;
+      v[8 * q + 2 * e + 1] = f.y;
+    }
+  }
 }
 
 // Bulk tensor store of a shared-memory block (tile mode; out-of-range parts are clipped).
@@ -360,13 +392,18 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
   constexpr bool kFuse = sizeof(AppT) > sizeof(TcNoApply);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int kStages = stages_for(PHASE);
+  constexpr uint32_t kWarpStage = warp_stage_bytes_for(PHASE);
+  constexpr uint32_t kOutPart = out_bytes_for(PHASE);
+  constexpr bool kHasIn = in_bytes_for(PHASE) > 0;
   uint8_t* out_stage = smem + kStages * kStageBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kOutBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kEpiWarps * kWarpStage);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* in_bar = drain + 1;  // [kEpiWarps][2] input-block barriers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(in_bar + 2 * kEpiWarps);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -385,6 +422,7 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
       mbar_init(&tempty[a], 2 * kEpiWarps);  // every epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
+    for (int b = 0; b < 2 * kEpiWarps; ++b) mbar_init(&in_bar[b], 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -499,14 +537,64 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
     const int quad = warp & 3;                       // TMEM lane quadrant this warp may access
-    uint8_t* my_stage = out_stage + (warp - 2) * kOutWarpBytes;
-    uint32_t n_out = 0;                              // staged blocks so far (buffer parity)
-    const int c_begin = ((warp - 2) / 4) * (kTile / 32 * 4 / kEpiWarps);  // first 32-column chunk
+    const int ew = warp - 2;                         // epilogue warp index
+    uint8_t* my_out = out_stage + ew * kWarpStage;   // [2] output buffers
+    uint8_t* my_in = my_out + kOutPart;              // [2] input buffers (Poly / Update)
+    uint64_t* my_bar = in_bar + 2 * ew;
+    constexpr int kChunks = kTile / 32 * 4 / kEpiWarps;
+    const int c_begin = (ew / 4) * kChunks;          // first 32-column chunk of this warp
     const uint32_t leader_tempty0 = peer_addr(smem_u32(&tempty[0]), 0);
+
+    // Valid chunks of a tile for this warp form the range [lo, hi): columns inside the
+    // result, and for Gram/Poly not strictly below the diagonal.
+    auto chunk_range = [&](const TcTile& tl, int& lo, int& hi) {
+      const TcGroup& gg = p.g[tl.group];
+      const int r0 = tl.bi * kTile + (int)rank * kHalf + 32 * quad;
+      lo = c_begin;
+      hi = c_begin + kChunks;
+      if (r0 >= gg.s) { hi = lo; return; }
+      const int lim = kSyrk ? gg.s : gg.L;
+      while (hi > lo && tl.bj * kTile + 32 * (hi - 1) >= lim) --hi;
+      if (kSyrk)
+        while (lo < hi && tl.bj * kTile + 32 * lo + 31 < r0) ++lo;
+    };
+    // Input prefetch cursor over (tile, chunk) pairs of this warp, in processing order:
+    // (pf_t, pf_c) is the next block to request; pf_t >= n_tiles when none is left.
+    int pf_t = p.n_tiles, pf_c = 0, pf_hi = 0;
+    uint32_t n_req = 0;  // input blocks requested so far (buffer = n & 1)
+    auto pf_first_from = [&](int t0) {  // first tile at or after t0 that has chunks for this warp
+      pf_t = t0;
+      while (pf_t < p.n_tiles) {
+        int lo, hi;
+        chunk_range(p.tiles[pf_t], lo, hi);
+        if (lo < hi) { pf_c = lo; pf_hi = hi; return; }
+        pf_t += n_clusters;
+      }
+    };
+    auto pf_issue = [&]() {  // lane 0 requests the cursor's block; every lane advances the cursor
+      if (pf_t >= p.n_tiles) return;
+      const TcTile tl = p.tiles[pf_t];
+      const int b = n_req & 1;
+      if (lane == 0) {
+        fence_async_smem();
+        mbar_arrive_expect_tx(&my_bar[b], kOutBlockBytes);
+        tma_load_3d_local(smem_u32(my_in + b * kOutBlockBytes), &p.map_in[tl.group], &my_bar[b],
+                          tl.bj * kTile + 32 * pf_c, tl.bi * kTile + (int)rank * kHalf + 32 * quad, tl.mat);
+      }
+      ++n_req;
+      if (++pf_c >= pf_hi) pf_first_from(pf_t + n_clusters);
+    };
+    if constexpr (kHasIn) {
+      pf_first_from(cluster);
+      pf_issue();
+    }
+    uint32_t n_used = 0;  // input blocks consumed so far
+    uint32_t n_out = 0;   // staged output blocks so far (buffer parity)
+
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int t = cluster; t < p.n_tiles; t += n_clusters) {
+    for (int t = cluster; t < p.n_tiles && ok; t += n_clusters) {
       const TcTile tile = p.tiles[t];
       const TcGroup& g = p.g[tile.group];
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) { ok = false; break; }
@@ -517,115 +605,88 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
       const int row = row0 + lane;
       const float sc = p.first_iter ? p.scale[g.gid_base + tile.mat] : 1.f;
       const uint32_t tbase = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(acc * kTile);
+      int c_lo, c_hi;
+      chunk_range(tile, c_lo, c_hi);
 
-      if (row0 < s) {
-        for (int c = c_begin; c < c_begin + kTile / 32 * 4 / kEpiWarps; ++c) {
-          const int col0 = tile.bj * kTile + 32 * c;
-          if (kSyrk) {
-            if (col0 >= s || col0 + 31 < row0) continue;  // outside / strictly lower block
-          } else {
-            if (col0 >= g.L) continue;
-          }
-          float v[32];
-          tmem_ld32(tbase + (uint32_t)(32 * c), v);
-          if (PHASE == kPhaseGram) {
-            const float alpha = sc * sc;
+      for (int c = c_lo; c < c_hi; ++c) {
+        const int col0 = tile.bj * kTile + 32 * c;
+        float in_v[32];
+        if constexpr (kHasIn) {
+          pf_issue();  // next block (this or a later tile) into the other buffer
+        }
+        float v[32];
+        tmem_ld32(tbase + (uint32_t)(32 * c), v);
+        if constexpr (kHasIn) {
+          const int b = n_used & 1;
+          if (!mbar_wait(&my_bar[b], (n_used >> 1) & 1u, abort_flag)) { ok = false; break; }
+          unstage_row(my_in + b * kOutBlockBytes, lane, in_v);
+          ++n_used;
+          __syncwarp();  // every lane has read the block before its buffer is refilled
+        }
+        if (PHASE == kPhaseGram) {
+          const float alpha = sc * sc;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= alpha;
-          } else if (PHASE == kPhasePoly) {
-            const __nv_bfloat16* a = g.gram + (size_t)tile.mat * s * g.ld_s;
-            if (row < s) {
-              float av[32];
-              if (col0 + 32 <= s) {
-                load_bf16x32(a + (size_t)row * g.ld_s + col0, av);
-              } else {
+          for (int j = 0; j < 32; ++j) v[j] *= alpha;
+        } else if (PHASE == kPhasePoly) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  av[j] = (col0 + j < s) ? __bfloat162float(a[(size_t)row * g.ld_s + col0 + j]) : 0.f;
-              }
+          for (int j = 0; j < 32; ++j) v[j] = fmaf(p.cb, in_v[j], p.cc * v[j]);
+        } else {
+          const float alpha = p.ca * sc;
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = fmaf(p.cb, av[j], p.cc * v[j]);
-            }
-          } else {
-            const size_t moff = (size_t)tile.mat * s * g.ld_x;
-            const __nv_bfloat16* x = g.x_cur + moff;
-            __nv_bfloat16* xn = g.x_next + moff;
-            const float alpha = p.ca * sc;
-            if constexpr (kFuse) {
-              if (row < s) {
-                float xv[32];
-                if (col0 + 32 <= g.L) {
-                  load_bf16x32(x + (size_t)row * g.ld_x + col0, xv);
-                } else {
-#pragma unroll
-                  for (int j = 0; j < 32; ++j)
-                    xv[j] = (col0 + j < g.L) ? __bfloat162float(x[(size_t)row * g.ld_x + col0 + j]) : 0.f;
-                }
-#pragma unroll
-                for (int j = 0; j < 32; ++j) xv[j] = fmaf(alpha, xv[j], sc * v[j]);
-                fused_apply_chunk(reinterpret_cast<const TcApplyTable&>(app).m[g.gid_base + tile.mat -
-                                                                                reinterpret_cast<const TcApplyTable&>(app).base],
-                                  s, g.L, row, col0, xv);
-              }
-              continue;
-            }
-            (void)xn;
-            float xv[32];
-            if (row < s && col0 + 32 <= g.L) {
-              load_bf16x32(x + (size_t)row * g.ld_x + col0, xv);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                xv[j] = (row < s && col0 + j < g.L) ? __bfloat162float(x[(size_t)row * g.ld_x + col0 + j]) : 0.f;
-            }
-#pragma unroll
-            for (int j = 0; j < 32; ++j) xv[j] = fmaf(alpha, xv[j], sc * v[j]);
-            uint8_t* blk = my_stage + (n_out & 1) * 2 * kOutBlockBytes;
-            if (lane == 0) bulk_wait_read_1();
-            __syncwarp();
-            stage_row(blk, lane, xv);
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_3d(&p.map_out[tile.group], smem_u32(blk), col0, row0, tile.mat);
-              bulk_commit();
-            }
-            ++n_out;
+          for (int j = 0; j < 32; ++j) v[j] = fmaf(alpha, in_v[j], sc * v[j]);
+          if constexpr (kFuse) {
+            if (row < s)
+              fused_apply_chunk(reinterpret_cast<const TcApplyTable&>(app).m[g.gid_base + tile.mat -
+                                                                              reinterpret_cast<const TcApplyTable&>(app).base],
+                                s, g.L, row, col0, v);
             continue;
           }
-          // symmetric store: the block (row0.., col0..) and its mirror (col0.., row0..),
-          // both built from the upper-triangle values so the result is exactly symmetric
-          uint8_t* blk = my_stage + (n_out & 1) * 2 * kOutBlockBytes;
+          uint8_t* blk = my_out + (n_out & 1) * kOutBlockBytes;
           if (lane == 0) bulk_wait_read_1();
           __syncwarp();
-          const bool upper = col0 >= row0 + 32;
-          if (upper) {
-            stage_row(blk, lane, v);
-            uint8_t* mir = blk + kOutBlockBytes;
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              *reinterpret_cast<__nv_bfloat16*>(mir + swz64(j, lane)) = __float2bfloat16_rn(v[j]);
-          } else {
-            // diagonal block (col0 == row0): element (lane, j) for j >= lane, mirrored below
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (j >= lane) {
-                const __nv_bfloat16 b = __float2bfloat16_rn(v[j]);
-                *reinterpret_cast<__nv_bfloat16*>(blk + swz64(lane, j)) = b;
-                if (j > lane) *reinterpret_cast<__nv_bfloat16*>(blk + swz64(j, lane)) = b;
-              }
-            }
-          }
+          stage_row(blk, lane, v);
           fence_async_smem();
           __syncwarp();
           if (lane == 0) {
             tma_store_3d(&p.map_out[tile.group], smem_u32(blk), col0, row0, tile.mat);
-            if (upper) tma_store_3d(&p.map_out[tile.group], smem_u32(blk + kOutBlockBytes), row0, col0, tile.mat);
             bulk_commit();
           }
           ++n_out;
+          continue;
         }
+        // symmetric store: the block (row0.., col0..) and its mirror (col0.., row0..),
+        // both built from the upper-triangle values so the result is exactly symmetric
+        uint8_t* blk = my_out + (n_out & 1) * 2 * kOutBlockBytes;
+        if (lane == 0) bulk_wait_read_1();
+        __syncwarp();
+        const bool upper = col0 >= row0 + 32;
+        if (upper) {
+          stage_row(blk, lane, v);
+          uint8_t* mir = blk + kOutBlockBytes;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            *reinterpret_cast<__nv_bfloat16*>(mir + swz64(j, lane)) = __float2bfloat16_rn(v[j]);
+        } else {
+          // diagonal block (col0 == row0): element (lane, j) for j >= lane, mirrored below
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (j >= lane) {
+              const __nv_bfloat16 bv = __float2bfloat16_rn(v[j]);
+              *reinterpret_cast<__nv_bfloat16*>(blk + swz64(lane, j)) = bv;
+              if (j > lane) *reinterpret_cast<__nv_bfloat16*>(blk + swz64(j, lane)) = bv;
+            }
+          }
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&p.map_out[tile.group], smem_u32(blk), col0, row0, tile.mat);
+          if (upper) tma_store_3d(&p.map_out[tile.group], smem_u32(blk + kOutBlockBytes), row0, col0, tile.mat);
+          bulk_commit();
+        }
+        ++n_out;
       }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) remote_arrive(leader_tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
@@ -637,6 +698,13 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
       atomicExch(p.status, kDevTimeout);
       *abort_flag = 1;
       remote_store_flag(peer_abort, 1);
+    }
+    if constexpr (kHasIn) {
+      // input blocks requested but not consumed (after an abort) land before exit
+      while (n_used < n_req) {
+        (void)mbar_wait(&my_bar[n_used & 1], (n_used >> 1) & 1u, nullptr);
+        ++n_used;
+      }
     }
   }
   (void)aborted;
@@ -656,7 +724,7 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
 template <int PHASE, typename AppT>
 cudaError_t set_smem_attr() {
   return cudaFuncSetAttribute(tc_kernel<PHASE, AppT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)kSmemBytes);
+                              (int)smem_bytes_for(PHASE));
 }
 
 struct DeviceInfo {
@@ -682,7 +750,7 @@ cudaError_t device_setup(int dev) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(sms & ~1), 1, 1);
   cfg.blockDim = dim3(kThreadsTc, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = smem_bytes_for(kPhaseUpdate);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -706,7 +774,7 @@ cudaError_t launch_phase(const TcParams& p, const AppT& app, int clusters, cudaS
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
   cfg.blockDim = dim3(kThreadsTc, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = smem_bytes_for(PHASE);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

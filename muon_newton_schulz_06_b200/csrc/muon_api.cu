@@ -509,10 +509,12 @@ muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, const s
           } else if (ph == kPhasePoly) {
             tp->map_a[li] = P.map_gram[gg];
             tp->map_out[li] = P.map_poly_out[gg];
+            tp->map_in[li] = P.map_gram_out[gg];
           } else {
             tp->map_a[li] = P.map_poly[gg];
             tp->map_b[li] = P.map_xmn[cur][gg];
             tp->map_out[li] = P.map_xout[cur ^ 1][gg];
+            tp->map_in[li] = P.map_xout[cur][gg];
           }
         }
         tp->tiles = reinterpret_cast<const TcTile*>(h->ws + P.off_tiles) + ch.off_tiles[ph];

@@ -102,6 +102,7 @@ struct __align__(64) TcParams {
   CUtensorMap map_a[kMaxGroups];    // A operand (K-major, box 64 x 128)
   CUtensorMap map_b[kMaxGroups];    // B operand (K-major box 64 x 128, or MN-major box 64 x 64)
   CUtensorMap map_out[kMaxGroups];  // output (X_next / Gram / Poly), box 32 x 32, 64-byte swizzle
+  CUtensorMap map_in[kMaxGroups];   // epilogue input (X_cur for Update, Gram for Poly), same boxes
   TcGroup g[kMaxGroups];
   const TcTile* tiles;
   int n_tiles;

@@ -197,10 +197,12 @@ extern "C" MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, voi
       } else if (ph == kPhasePoly) {
         g_tc.map_a[0] = gram_map;
         g_tc.map_out[0] = poly_out;
+        g_tc.map_in[0] = gram_out;
       } else {
         g_tc.map_a[0] = poly_map;
         g_tc.map_b[0] = xmn[cur];
         g_tc.map_out[0] = xout[cur ^ 1];
+        g_tc.map_in[0] = xout[cur];
       }
       g_tc.tiles = ph == kPhaseUpdate ? dev_tiles + n_syrk : dev_tiles;
       g_tc.n_tiles = ph == kPhaseUpdate ? n_upd : n_syrk;
