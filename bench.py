@@ -69,6 +69,26 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def measured_traffic(config, layers):
+    """DRAM bytes per launch of each kernel kind from the committed ncu summary, or {}
+    when the kernel sources have changed since the capture (or for another workload)."""
+    import glob
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "ncu_traffic_llama3p8b.json")
+    if config != 4 or layers or not os.path.exists(path):
+        return {}
+    with open(path) as f:
+        t = json.load(f)
+    files = sorted(glob.glob(os.path.join(ROOT, "muon_newton_schulz_06_b200", "csrc", "*.cu")) +
+                   glob.glob(os.path.join(ROOT, "muon_newton_schulz_06_b200", "csrc", "*.h")))
+    h = hashlib.sha256()
+    for fn in files:
+        h.update(os.path.basename(fn).encode())
+        with open(fn, "rb") as fh:
+            h.update(fh.read())
+    return t["per_full_launch_bytes"] if h.hexdigest() == t.get("csrc_sha256") else {}
+
+
 # ------------------------------------------------------------------ clocks during the timed region
 
 class ClockSampler:
@@ -318,6 +338,7 @@ def main():
 
     # ---------------- per-kernel roofline
     pk = peaks()
+    traffic = measured_traffic(cfg, args.layers)
     kernels = {}
     for kind, (kms, n) in prof.items():
         if n == 0:
@@ -335,13 +356,16 @@ def main():
             kernels[kind] = {"bound": "hbm", "ms_per_launch": avg_ms, "launches": n, "achieved": ach,
                              "unit": "GB/s", "work_per_launch": work, "frac": ach / pk["hbm_gbs"]}
         kernels[kind]["share"] = kms / max(sum(v[0] for v in prof.values()), 1e-9)
+        kernels[kind]["traffic"] = traffic.get(kind)
     dom = max(kernels, key=lambda k: kernels[k]["share"])
     dk = kernels[dom]
     roofline = {"bound": dk["bound"], "kernel": dom, "achieved": dk["achieved"],
                 "peak": pk["bf16_tflops_sustained"] if dk["bound"] == "tensor" else pk["hbm_gbs"],
                 "peak_kind": ("sustained bf16 (kernel timed inside a long loop), " if dk["bound"] == "tensor"
                               else "copy bandwidth, ") + pk["source"],
-                "unit": dk["unit"], "frac": dk["frac"], "traffic": None}
+                "unit": dk["unit"], "frac": dk["frac"], "traffic": dk["traffic"],
+                "traffic_note": "DRAM bytes per launch (ncu, first layer x 28 layers); null if the kernels "
+                                "changed since the capture"}
     ns_ms = sum(prof[k][0] for k in ("gram", "poly", "update", "update_apply")) / args.steps
     ns_tflops = fl["algorithmic"] / (ns_ms / 1e3) / 1e12 if ns_ms > 0 else None
 
