@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--layers", type=int, default=0,
                     help="keep only the first N layers of the set (profiling captures); 0 = all")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--shard", action="store_true",
+                    help="split the matrices across ranks (strong scaling, one all-gather of the new "
+                         "weights per step) instead of running one replica per rank")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
@@ -267,9 +270,19 @@ def main():
 
     h = mb.muon_init(local)
     stream = torch.cuda.current_stream(dev)
+    if args.shard:
+        from muon_newton_schulz_06_b200.sharded import ShardedMuon
+        sm = ShardedMuon(W, device=dev, handle=h)
+        W = sm.params
+        del M
 
-    def step():
-        mb.muon_step(h, W, G, M, lr=LR, momentum=MU, nesterov=True, ns_steps=NS_STEPS, eps=EPS, stream=stream)
+        def step():
+            sm.step(G, lr=LR, momentum=MU, nesterov=True, ns_steps=NS_STEPS, eps=EPS, stream=stream)
+    else:
+        sm = None
+
+        def step():
+            mb.muon_step(h, W, G, M, lr=LR, momentum=MU, nesterov=True, ns_steps=NS_STEPS, eps=EPS, stream=stream)
 
     for _ in range(max(args.warmup, 0)):
         step()
@@ -309,7 +322,8 @@ def main():
     prof = mb.muon_profile_read(h)
     mb.muon_profile_enable(h, False)
     ms_max = max_over_ranks(ms, world, dev)
-    value = replica_throughput(fl["algorithmic"], args.steps, world, ms_max)
+    # replicas: every rank does the whole set; sharded: the ranks share one set
+    value = replica_throughput(fl["algorithmic"], args.steps, 1 if args.shard else world, ms_max)
 
     # ---------------- end to end: pinned host gradients in, updated weights out, every step
     e2e = None
@@ -332,7 +346,8 @@ def main():
         e3.record(stream)
         torch.cuda.synchronize()
         ms_e2e = max_over_ranks(e2.elapsed_time(e3), world, dev)
-        e2e = {"value": replica_throughput(fl["algorithmic"], args.steps, world, ms_e2e), "unit": UNIT,
+        e2e = {"value": replica_throughput(fl["algorithmic"], args.steps, 1 if args.shard else world, ms_e2e),
+               "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / args.steps}
         del g_host, w_host
 
@@ -381,7 +396,8 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "strong" if args.shard else "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
             "config": {"workload": WORKLOAD_TEXT[cfg] + (f" (first {args.layers} layers only)" if args.layers
                                                           else ""), "matrices": len(shapes),
                        "params": int(eb["numel"]), "ns_steps": NS_STEPS,
@@ -389,13 +405,14 @@ def main():
                        "nesterov": True, "eps": EPS,
                        "l2": "no flush: inputs larger than L2 (%.1f GB of gradients per step)" % (
                            sum(g.numel() * g.element_size() for g in G) / 1e9),
-                       "parallelism": "replicas" if world > 1 else "single GPU"},
+                       "parallelism": ("matrix-sharded, all-gather of new weights" if args.shard else
+                                       "replicas" if world > 1 else "single GPU")},
             "ns_tflops_algorithmic": ns_tflops,
             "ns_frac_of_sustained_peak": ns_tflops / pk["bf16_tflops_sustained"] if ns_tflops else None,
             "ns_frac_of_burst_peak": ns_tflops / pk["bf16_tflops"] if ns_tflops else None,
             "ns_tflop_per_step_algorithmic": fl["algorithmic"] / 1e12,
             "ns_tflop_per_step_dense_equivalent": fl["dense_equivalent"] / 1e12,
-            "matrices_per_s": len(shapes) * args.steps * world / (ms_max / 1e3),
+            "matrices_per_s": len(shapes) * args.steps * (1 if args.shard else world) / (ms_max / 1e3),
             "kernels": kernels, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
         }

@@ -67,3 +67,64 @@ def test_reference_arm_runs_on_rank_zero_only():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
                         "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+# ---------------------------------------------------------------- matrix-sharded step (host logic)
+
+from muon_newton_schulz_06_b200 import sharded  # noqa: E402
+import synth  # noqa: E402
+
+
+def test_lpt_partition_balances_the_llama_set():
+    shapes = [(s.rows, s.cols) for s in synth.config_shapes(4)]
+    from muon_newton_schulz_06_b200.cost import ns_flops
+    for world in (1, 2, 4, 8):
+        owner = sharded.partition_lpt(shapes, world)
+        assert sorted(set(owner)) == list(range(world))
+        loads = [sum(ns_flops([shapes[i]])["algorithmic"] for i in range(len(shapes)) if owner[i] == r)
+                 for r in range(world)]
+        assert max(loads) / (sum(loads) / world) < 1.03, (world, loads)
+    assert sharded.partition_lpt(shapes, 3) == sharded.partition_lpt(shapes, 3)  # deterministic
+
+
+def _fake_step(params, grads, moms, lr=0.1, **kw):
+    # stands in for the CUDA step on CPU: any deterministic in-place update will do
+    for w, g, m in zip(params, grads, moms):
+        m.mul_(0.5).add_(g.float())
+        w.sub_(lr * m.to(w.dtype))
+
+
+def _sharded_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=30))
+    try:
+        shapes = [(6, 4), (4, 6), (8, 8), (10, 3), (3, 10), (5, 5), (12, 12)]
+        gen = torch.Generator().manual_seed(0)
+        params = [torch.randn(r, c, generator=gen) for r, c in shapes]      # same on every rank
+        grads = [torch.randn(r, c, generator=gen) for r, c in shapes]
+        sm = sharded.ShardedMuon(params, device="cpu", step_fn=_fake_step)
+        for _ in range(3):
+            sm.step([g if sm.owner[i] == rank else None for i, g in enumerate(grads)], lr=0.1)
+        out[rank] = ([p.clone() for p in sm.params], sm.owner, sorted(sm.moms))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_step_gives_every_rank_the_same_updated_weights():
+    world = 2
+    out = mp.Manager().dict()
+    mp.spawn(_sharded_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+    # reference: the same fake step on every matrix in one process
+    shapes = [(6, 4), (4, 6), (8, 8), (10, 3), (3, 10), (5, 5), (12, 12)]
+    gen = torch.Generator().manual_seed(0)
+    params = [torch.randn(r, c, generator=gen) for r, c in shapes]
+    grads = [torch.randn(r, c, generator=gen) for r, c in shapes]
+    moms = [torch.zeros(r, c) for r, c in shapes]
+    for _ in range(3):
+        _fake_step(params, grads, moms, lr=0.1)
+    for r in range(world):
+        got, owner, mine = out[r]
+        for a, b in zip(got, params):
+            assert torch.equal(a, b)
+        assert mine == [i for i in range(len(shapes)) if owner[i] == r]  # momentum only where owned
