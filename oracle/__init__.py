@@ -31,4 +31,5 @@ from .muon import (  # noqa: F401
     update_scale,
     muon_step_matrix,
     muon_step,
+    cautious_mask,
 )

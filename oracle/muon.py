@@ -30,7 +30,11 @@ design notes of the library):
 * The per-step coefficient table is an input; the page says the values are
   precomputed ("Polar Express") but prints none.  ``QUINTIC`` repeated five times
   is the default.
-* No weight decay on this path.
+* Weight decay is optional (default off): W -= lr*wd*W on every entry, or only where
+  the update and the parameter agree in sign (cautious decay; the page gives the mask
+  (g x parameter) >= 0, read with g = O, the update that is applied).
+* The interpolation form of the momentum (M <- mu*M + (1-mu)*G) is an option next to
+  the default SGD form.
 """
 from __future__ import annotations
 
@@ -46,19 +50,29 @@ QUINTIC = (3.4445, -4.7750, 2.0315)
 CUBIC = (1.5, -0.5, 0.0)
 
 
-def nesterov_momentum_f32(grad, momentum, mu: float, nesterov: bool = True):
+def nesterov_momentum_f32(grad, momentum, mu: float, nesterov: bool = True, lerp: bool = False):
     """Momentum step on the float32 buffer (autoresearch review, MuonAdamW paragraph:
     Muon applies Nesterov momentum to the gradient; the buffer has the parameter's
     shape).
 
-    Returns (M_new float32, U float64).  M_new = fl32(fl32(mu*M) + G): NumPy float32
-    arithmetic rounds the product and the sum separately.  U = G + mu*M_new for
-    Nesterov, else M_new, evaluated in float64 from the float32 values.
+    Returns (M_new float32, U float64).  SGD form (default): M_new = fl32(fl32(mu*M) + G),
+    U = G + mu*M_new for Nesterov, else M_new.  Interpolation ("lerp") form:
+    M_new = fl32(fl32(mu*M) + fl32((1-mu)*G)), U = (1-mu)*G + mu*M_new for Nesterov, else
+    M_new, with 1-mu rounded to float32 once.  NumPy float32 arithmetic rounds every
+    product and sum separately; U is evaluated in float64 from the float32 values.
     """
     g32 = np.asarray(grad, dtype=np.float32)
     m32 = np.asarray(momentum, dtype=np.float32)
     mu32 = np.float32(mu)
     prod = np.multiply(mu32, m32, dtype=np.float32)
+    if lerp:
+        omu = np.float32(np.float32(1.0) - mu32)
+        m_new = np.add(prod, np.multiply(omu, g32, dtype=np.float32), dtype=np.float32)
+        if nesterov:
+            u = np.float64(omu) * g32.astype(np.float64) + np.float64(mu32) * m_new.astype(np.float64)
+        else:
+            u = m_new.astype(np.float64)
+        return m_new, u
     m_new = np.add(prod, g32, dtype=np.float32)
     if nesterov:
         u = g32.astype(np.float64) + np.float64(mu32) * m_new.astype(np.float64)
@@ -103,21 +117,32 @@ def update_scale(rows: int, cols: int) -> float:
     return math.sqrt(max(1.0, rows / cols))
 
 
+def cautious_mask(o, w):
+    """Cautious weight decay (autoresearch review, MuonAdamW paragraph): only entries whose
+    update and parameter agree in sign decay, mask = (O * W) >= 0 (zeros included)."""
+    return (np.asarray(o, dtype=np.float64) * np.asarray(w, dtype=np.float64)) >= 0
+
+
 def muon_step_matrix(w, grad, momentum, *, lr: float, mu: float, nesterov: bool = True,
-                     coeffs: Sequence[Sequence[float]] | None = None, eps: float = 1e-7):
+                     coeffs: Sequence[Sequence[float]] | None = None, eps: float = 1e-7,
+                     lerp: bool = False, weight_decay: float = 0.0, cautious: bool = False):
     """One Muon step for one matrix.
 
     Returns (W_new float64, M_new float32, O float64).  W_new is the exact
-    W - lr*scale*O; rounding it to the parameter's dtype is the caller's concern.
+    W - lr*scale*O - lr*weight_decay*mask*W with mask = 1 everywhere, or the cautious
+    mask when ``cautious``; rounding to the parameter's dtype is the caller's concern.
     """
     if coeffs is None:
         coeffs = [QUINTIC] * 5
     w64 = np.asarray(w, dtype=np.float64)
     rows, cols = w64.shape
-    m_new, u = nesterov_momentum_f32(grad, momentum, mu, nesterov)
+    m_new, u = nesterov_momentum_f32(grad, momentum, mu, nesterov, lerp=lerp)
     x0 = frobenius_normalise(u, eps)
     o = newton_schulz(x0, coeffs)
     w_new = w64 - lr * update_scale(rows, cols) * o
+    if weight_decay:
+        mask = cautious_mask(o, w64) if cautious else np.ones_like(w64, dtype=bool)
+        w_new = w_new - lr * weight_decay * np.where(mask, w64, 0.0)
     return w_new, m_new, o
 
 

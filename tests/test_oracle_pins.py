@@ -303,3 +303,45 @@ def test_pins_catch_planted_mistakes(kind):
         except (AssertionError, ValueError):
             caught += 1
     assert caught >= 1, kind
+
+
+# ---------------------------------------------------------------- options: lerp momentum, weight decay
+
+def test_lerp_momentum_closed_form():
+    """Interpolation form from M = 0 with a constant gradient: M_k = g (1 - mu^k),
+    U_k = (1 - mu) g + mu M_k; exact small case with mu = 0.5."""
+    mu = 0.75
+    g = np.full(6, 0.5, np.float32)
+    m = np.zeros(6, np.float32)
+    for k in range(1, 25):
+        m, u = oracle.nesterov_momentum_f32(g, m, mu, True, lerp=True)
+        mk = 0.5 * (1 - 0.75 ** k)
+        assert np.allclose(m, mk, rtol=1e-6)
+        assert np.allclose(u, 0.25 * 0.5 + 0.75 * mk, rtol=1e-6)
+    m2, u2 = oracle.nesterov_momentum_f32(np.array([1.0, -2.0], np.float32), np.array([4.0, 2.0], np.float32),
+                                         0.5, True, lerp=True)
+    assert np.array_equal(m2, np.array([2.5, 0.0], np.float32))
+    assert np.array_equal(u2, np.array([1.75, -1.0]))
+
+
+def test_weight_decay_and_cautious_mask_closed_form():
+    """Diagonal gradient: O is diagonal with the scalar map's (positive) values and zero
+    elsewhere, so the cautious mask (O * W >= 0) is false only where a diagonal entry
+    of W is negative; the decayed weights are worked out by hand."""
+    g = np.diag([0.8, 0.6, 0.3]).astype(np.float32)
+    w = np.array([[0.5, -0.2, 0.1], [0.3, -0.4, -0.6], [-0.7, 0.2, 0.9]])
+    z = np.zeros((3, 3), np.float32)
+    coeffs = [QUINTIC] * 5
+    w_plain, _, o = oracle.muon_step_matrix(w, g, z, lr=0.1, mu=0.0, coeffs=coeffs, eps=0.0)
+    d = np.array([0.8, 0.6, 0.3]) / np.linalg.norm([0.8, 0.6, 0.3])
+    od = scalar_map(d, coeffs)
+    assert np.allclose(o, np.diag(od), atol=1e-15) and np.all(od > 0)
+    # O is zero off the diagonal (mask true there), positive on it (mask = W >= 0)
+    mask = np.ones((3, 3), bool)
+    mask[1, 1] = False  # W[1,1] = -0.4 < 0 while O[1,1] > 0
+    assert np.array_equal(oracle.cautious_mask(o, w), mask)
+    w_cwd, _, _ = oracle.muon_step_matrix(w, g, z, lr=0.1, mu=0.0, coeffs=coeffs, eps=0.0, weight_decay=0.5,
+                                          cautious=True)
+    assert np.allclose(w_cwd, w - 0.1 * np.diag(od) - 0.05 * np.where(mask, w, 0.0), atol=1e-15)
+    w_wd, _, _ = oracle.muon_step_matrix(w, g, z, lr=0.1, mu=0.0, coeffs=coeffs, eps=0.0, weight_decay=0.5)
+    assert np.allclose(w_wd, w_plain - 0.05 * w, atol=1e-15)
