@@ -112,6 +112,40 @@ MUON_API muon_status muon_step(muon_handle_t h, const muon_matrix* mats, int n,
                       const float* coeffs, int ns_steps, float eps,
                       muon_mode mode, void* cuda_stream);
 
+/* Form of the momentum buffer update. */
+typedef enum {
+  MUON_MOMENTUM_SGD = 0,  /* M <- fl32(fl32(mu*M) + G);  Nesterov U = fl32(G + fl32(mu*M)) */
+  MUON_MOMENTUM_LERP = 1  /* M <- fl32(fl32(mu*M) + fl32((1-mu)*G));
+                             Nesterov U = fl32(fl32((1-mu)*G) + fl32(mu*M)); 1-mu in float32 */
+} muon_momentum_form;
+
+/* All options of one step (muon_step_ex).  Fields as in muon_step, plus:
+ *  momentum_form   MUON_MOMENTUM_SGD (muon_step's form) or MUON_MOMENTUM_LERP
+ *  weight_decay    >= 0; 0 disables.  W <- fl32(W' - fl32(fl32(lr*wd)*W)) after the
+ *                  update W' = fl32(W - fl32(lr*scale)*O), with W the weight before the
+ *                  step
+ *  cautious        nonzero: decay only entries where O*W >= 0 (update and weight agree
+ *                  in sign; zeros count as agreeing) -- the cautious weight decay of the
+ *                  autoresearch train.py review's MuonAdamW paragraph */
+typedef struct {
+  float lr;
+  float momentum;
+  int nesterov;
+  muon_momentum_form momentum_form;
+  const float* coeffs;
+  int ns_steps;
+  float eps;
+  muon_mode mode;
+  float weight_decay;
+  int cautious;
+} muon_options;
+
+/* muon_step with every option; `opt` is a HOST pointer.  muon_step(h, mats, n, lr, mu,
+ * nesterov, coeffs, ns_steps, eps, mode, stream) equals muon_step_ex with
+ * momentum_form = MUON_MOMENTUM_SGD, weight_decay = 0, cautious = 0. */
+MUON_API muon_status muon_step_ex(muon_handle_t h, const muon_matrix* mats, int n,
+                                  const muon_options* opt, void* cuda_stream);
+
 /* Newton-Schulz part alone: o_out[i] = X_K of X0 = x_in[i] / (||x_in[i]||_F + eps)
  * for n matrices of shape rows[i] x cols[i].  x_in and o_out are DEVICE pointers
  * of `dtype`; o_out must not overlap any input.  rows, cols, x_in and o_out are

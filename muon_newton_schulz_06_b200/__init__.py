@@ -32,7 +32,8 @@ MUON_BF16 = 1
 MUON_MODE_BF16 = 0
 MUON_MODE_FP32_VALIDATE = 1
 
-EXPORTED = ("muon_init", "muon_step", "muon_newton_schulz", "muon_newton_schulz_noalloc", "muon_sync",
+EXPORTED = ("muon_init", "muon_step", "muon_step_ex", "muon_newton_schulz", "muon_newton_schulz_noalloc",
+            "muon_sync",
             "muon_selftest_wait_timeout", "muon_workspace_bytes",
             "muon_last_launch_count", "muon_profile_enable", "muon_profile_read", "muon_destroy",
             "muon_status_string", "muon_last_error")
@@ -53,6 +54,17 @@ class muon_matrix(ctypes.Structure):
                 ("param_dtype", ctypes.c_int), ("grad_dtype", ctypes.c_int)]
 
 
+MUON_MOMENTUM_SGD = 0
+MUON_MOMENTUM_LERP = 1
+
+
+class muon_options(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("momentum", ctypes.c_float), ("nesterov", ctypes.c_int),
+                ("momentum_form", ctypes.c_int), ("coeffs", ctypes.POINTER(ctypes.c_float)),
+                ("ns_steps", ctypes.c_int), ("eps", ctypes.c_float), ("mode", ctypes.c_int),
+                ("weight_decay", ctypes.c_float), ("cautious", ctypes.c_int)]
+
+
 _lib_handle = None
 
 
@@ -70,6 +82,8 @@ def load_library(path: str = LIB_PATH):
     lib.muon_step.argtypes = [vp, ctypes.POINTER(muon_matrix), i32, f32, f32, i32, ctypes.POINTER(f32), i32,
                               f32, i32, vp]
     lib.muon_step.restype = i32
+    lib.muon_step_ex.argtypes = [vp, ctypes.POINTER(muon_matrix), i32, ctypes.POINTER(muon_options), vp]
+    lib.muon_step_ex.restype = i32
     lib.muon_newton_schulz.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(i64),
                                        ctypes.POINTER(i64), i32, i32, ctypes.POINTER(f32), i32, f32, i32, vp]
     lib.muon_newton_schulz.restype = i32
@@ -153,11 +167,7 @@ def muon_init(device: int = 0):
     return h
 
 
-def muon_step(handle, params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
-              moms: Sequence[torch.Tensor], lr: float, momentum: float = 0.95, nesterov: bool = True,
-              coeffs=None, ns_steps: int = 5, eps: float = 1e-7, mode="bf16", stream=None) -> None:
-    """One Muon step over matched lists of parameters (bf16/fp32, updated in place),
-    gradients (bf16/fp32) and float32 momentum buffers (updated in place)."""
+def _matrix_array(params, grads, moms):
     n = len(params)
     if len(grads) != n or len(moms) != n:
         raise ValueError("params, grads and moms must have the same length")
@@ -172,11 +182,37 @@ def muon_step(handle, params: Sequence[torch.Tensor], grads: Sequence[torch.Tens
             raise ValueError(f"matrix {i}: param, grad and momentum shapes differ")
         arr[i] = muon_matrix(w.data_ptr(), g.data_ptr(), m.data_ptr(), w.shape[0], w.shape[1],
                              _dtype_code(w), _dtype_code(g))
+    return arr, n
+
+
+def muon_step(handle, params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
+              moms: Sequence[torch.Tensor], lr: float, momentum: float = 0.95, nesterov: bool = True,
+              coeffs=None, ns_steps: int = 5, eps: float = 1e-7, mode="bf16", stream=None) -> None:
+    """One Muon step over matched lists of parameters (bf16/fp32, updated in place),
+    gradients (bf16/fp32) and float32 momentum buffers (updated in place)."""
+    arr, n = _matrix_array(params, grads, moms)
     dev = params[0].device if n else torch.device("cuda")
     c = _coeff_array(coeffs, ns_steps)
     _check(load_library().muon_step(handle, arr, n, float(lr), float(momentum), 1 if nesterov else 0, c,
                                     int(ns_steps), float(eps), _mode_code(mode), _stream_ptr(stream, dev)),
            handle)
+
+
+def muon_step_ex(handle, params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
+                 moms: Sequence[torch.Tensor], lr: float, momentum: float = 0.95, nesterov: bool = True,
+                 momentum_form: str = "sgd", coeffs=None, ns_steps: int = 5, eps: float = 1e-7, mode="bf16",
+                 weight_decay: float = 0.0, cautious: bool = False, stream=None) -> None:
+    """muon_step with every option: momentum_form "sgd" or "lerp"; weight_decay (0 = off);
+    cautious (decay only where the update and the weight agree in sign)."""
+    forms = {"sgd": MUON_MOMENTUM_SGD, "lerp": MUON_MOMENTUM_LERP}
+    if momentum_form not in forms:
+        raise ValueError(f"unknown momentum_form {momentum_form!r}")
+    arr, n = _matrix_array(params, grads, moms)
+    dev = params[0].device if n else torch.device("cuda")
+    c = _coeff_array(coeffs, ns_steps)
+    opt = muon_options(float(lr), float(momentum), 1 if nesterov else 0, forms[momentum_form], c, int(ns_steps),
+                       float(eps), _mode_code(mode), float(weight_decay), 1 if cautious else 0)
+    _check(load_library().muon_step_ex(handle, arr, n, ctypes.byref(opt), _stream_ptr(stream, dev)), handle)
 
 
 def muon_newton_schulz(handle, xs: Sequence[torch.Tensor], outs: Sequence[torch.Tensor], coeffs=None,
@@ -270,7 +306,7 @@ class Muon:
         self.handle = muon_init(device)
 
     def step(self, params, grads, moms, **kw):
-        muon_step(self.handle, params, grads, moms, **kw)
+        muon_step_ex(self.handle, params, grads, moms, **kw)
 
     def newton_schulz(self, xs, outs, **kw):
         muon_newton_schulz(self.handle, xs, outs, **kw)

@@ -6,8 +6,9 @@
 //    1/(||U||_F + eps).  Autoresearch train.py review, MuonAdamW paragraph: Muon
 //    applies Nesterov momentum to the gradient with a buffer of the parameter's shape;
 //    the Frobenius normalisation is the benchmark spec's.
-//  * apply: W <- fl32(W - lrs*O) rounded to the parameter dtype, O read back from the
-//    workspace (transposed for tall matrices); or export O into a caller buffer.
+//  * apply: W <- fl32(W - lrs*O) (then, with weight decay, - fl32(lr*wd)*W_old where the
+//    decay applies) rounded to the parameter dtype, O read back from the workspace
+//    (transposed for tall matrices); or export O into a caller buffer.
 //
 // One work unit is a 64 x 64 tile of the caller matrix; 256 threads each own 2 rows x 8
 // consecutive columns, so rows move as 16-byte vectors (streaming cache hints: every
@@ -142,9 +143,10 @@ momentum_norm_kernel(const __grid_constant__ EwParams p) {
       if (p.use_momentum) {
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          const float mn = __fadd_rn(__fmul_rn(p.mu, mo[pr][q]), g[pr][q]);
+          const float gq = p.lerp ? __fmul_rn(p.omu, g[pr][q]) : g[pr][q];
+          const float mn = __fadd_rn(__fmul_rn(p.mu, mo[pr][q]), gq);
           mo[pr][q] = mn;
-          g[pr][q] = p.nesterov ? __fadd_rn(g[pr][q], __fmul_rn(p.mu, mn)) : mn;  // g now holds U
+          g[pr][q] = p.nesterov ? __fadd_rn(gq, __fmul_rn(p.mu, mn)) : mn;  // g now holds U
         }
       }
 #pragma unroll
@@ -305,7 +307,13 @@ apply_kernel(const __grid_constant__ EwParams p, int out_kind) {
       const size_t base = (size_t)r * m.cols + c;
       if (out_kind == kEwApply) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) w[pr][q] = __fsub_rn(w[pr][q], __fmul_rn(m.lrs, o[pr][q]));
+        for (int q = 0; q < 8; ++q) {
+          const float w0 = w[pr][q], oq = o[pr][q];
+          float wn = __fsub_rn(w0, __fmul_rn(m.lrs, oq));
+          const bool agree = (oq >= 0.f && w0 >= 0.f) || (oq <= 0.f && w0 <= 0.f);
+          if (m.lrwd != 0.f && (!p.cautious || agree)) wn = __fsub_rn(wn, __fmul_rn(m.lrwd, w0));
+          w[pr][q] = wn;
+        }
       } else {
 #pragma unroll
         for (int q = 0; q < 8; ++q) w[pr][q] = o[pr][q];

@@ -323,9 +323,17 @@ struct TcNoApply {
 // Weight update of one 32-column chunk of a fused epilogue (see TcApply).  xv holds
 // X_K in fp32; O is its bf16 rounding, as the workspace copy would hold it.  All 32
 // weight loads of the chunk are issued before any store.
+// New weight of one entry: fl32(W - lrs*O), then weight decay where it applies.
+__device__ __forceinline__ float apply_one(float w0, float o, float lrs, float lrwd, bool cautious) {
+  float wn = __fsub_rn(w0, __fmul_rn(lrs, o));
+  const bool agree = (o >= 0.f && w0 >= 0.f) || (o <= 0.f && w0 <= 0.f);
+  if (lrwd != 0.f && (!cautious || agree)) wn = __fsub_rn(wn, __fmul_rn(lrwd, w0));
+  return wn;
+}
+
 template <typename WT>
-__device__ __forceinline__ void fused_apply_chunk_t(WT* w, float lrs, bool transposed, bool vec, int s, int L,
-                                                    int row, int col0, const float* xv) {
+__device__ __forceinline__ void fused_apply_chunk_t(WT* w, float lrs, float lrwd, bool cautious, bool transposed,
+                                                    bool vec, int s, int L, int row, int col0, const float* xv) {
   float o[32], wv[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) o[j] = __bfloat162float(__float2bfloat16_rn(xv[j]));
@@ -342,8 +350,13 @@ __device__ __forceinline__ void fused_apply_chunk_t(WT* w, float lrs, bool trans
         wv[4 * q] = v.x; wv[4 * q + 1] = v.y; wv[4 * q + 2] = v.z; wv[4 * q + 3] = v.w;
       }
     }
+    if (lrwd == 0.f) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) wv[j] = __fsub_rn(wv[j], __fmul_rn(lrs, o[j]));
+      for (int j = 0; j < 32; ++j) wv[j] = __fsub_rn(wv[j], __fmul_rn(lrs, o[j]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) wv[j] = apply_one(wv[j], o[j], lrs, lrwd, cautious);
+    }
     if constexpr (sizeof(WT) == 2) {
       store_bf16x32(reinterpret_cast<__nv_bfloat16*>(p), wv);
     } else {
@@ -367,10 +380,17 @@ __device__ __forceinline__ void fused_apply_chunk_t(WT* w, float lrs, bool trans
     }
     wv[j] = x;
   }
+  if (lrwd == 0.f) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) wv[j] = __fsub_rn(wv[j], __fmul_rn(lrs, o[j]));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) wv[j] = apply_one(wv[j], o[j], lrs, lrwd, cautious);
+  }
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
     if (col0 + j < L) {
-      const float r = __fsub_rn(wv[j], __fmul_rn(lrs, o[j]));
+      const float r = wv[j];
       if constexpr (sizeof(WT) == 2) p0[j * stride] = __float2bfloat16_rn(r);
       else p0[j * stride] = r;
     }
@@ -379,11 +399,11 @@ __device__ __forceinline__ void fused_apply_chunk_t(WT* w, float lrs, bool trans
 
 __device__ __forceinline__ void fused_apply_chunk(const TcApply& ap, int s, int L, int row, int col0,
                                                   const float* xv) {
-  const bool tr = ap.flags & kApplyTransposed, vec = ap.flags & kApplyVec;
+  const bool tr = ap.flags & kApplyTransposed, vec = ap.flags & kApplyVec, ca = ap.flags & kApplyCautious;
   if (ap.flags & kApplyBf16)
-    fused_apply_chunk_t(reinterpret_cast<__nv_bfloat16*>(ap.w), ap.lrs, tr, vec, s, L, row, col0, xv);
+    fused_apply_chunk_t(reinterpret_cast<__nv_bfloat16*>(ap.w), ap.lrs, ap.lrwd, ca, tr, vec, s, L, row, col0, xv);
   else
-    fused_apply_chunk_t(reinterpret_cast<float*>(ap.w), ap.lrs, tr, vec, s, L, row, col0, xv);
+    fused_apply_chunk_t(reinterpret_cast<float*>(ap.w), ap.lrs, ap.lrwd, ca, tr, vec, s, L, row, col0, xv);
 }
 
 template <int PHASE, typename AppT>

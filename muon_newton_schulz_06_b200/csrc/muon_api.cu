@@ -379,7 +379,20 @@ struct CallMat {
   float* mom;
   void* out;          // o_out (Newton-Schulz entry)
   bool param_bf16, grad_bf16;
-  float lrs;
+  float lrs;          // fl32(lr * sqrt(max(1, rows/cols)))
+  float lrwd;         // fl32(lr * weight_decay)
+};
+
+// Per-call options shared by every matrix.
+struct CallOpts {
+  float mu = 0.f;
+  int nesterov = 0;
+  int lerp = 0;
+  int cautious = 0;
+  const float* coeffs = nullptr;
+  int ns_steps = 5;
+  float eps = 0.f;
+  muon_mode mode = MUON_MODE_BF16;
 };
 
 void* work_ptr(muon_handle* h, const MatPlan& m, int buf) {
@@ -390,7 +403,9 @@ void* work_ptr(muon_handle* h, const MatPlan& m, int buf) {
 }
 
 muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, bool momentum_pass,
-                               int out_kind, int work_buf, float mu, int nesterov, float eps, cudaStream_t st) {
+                               int out_kind, int work_buf, const CallOpts& o, cudaStream_t st) {
+  const float mu = o.mu, eps = o.eps;
+  const int nesterov = o.nesterov;
   const Plan& P = h->plan;
   const int n = (int)cm.size();
   const bool f32 = (P.mode == MUON_MODE_FP32_VALIDATE);
@@ -401,6 +416,9 @@ muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, b
     ep->mu = mu;
     ep->nesterov = nesterov;
     ep->use_momentum = (momentum_pass && cm[b].mom != nullptr) ? 1 : 0;
+    ep->lerp = o.lerp;
+    ep->omu = 1.0f - mu;
+    ep->cautious = o.cautious;
     ep->eps = eps;
     ep->partials = reinterpret_cast<float*>(h->ws + P.off_partials);
     ep->scale = reinterpret_cast<float*>(h->ws + P.off_scale);
@@ -428,6 +446,7 @@ muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, b
       e.param_bf16 = cm[i].param_bf16 ? 1 : 0;
       e.grad_bf16 = cm[i].grad_bf16 ? 1 : 0;
       e.lrs = cm[i].lrs;
+      e.lrwd = cm[i].lrwd;
       units += m.n_units;
     }
     ep->total_units = units;
@@ -456,7 +475,7 @@ bool can_fuse_apply(const Plan& P) {
 // fuse_cm: caller matrices whose weight update is fused into the last Update pass
 // (nullptr: the last pass stores X_K for a separate apply / export pass).
 muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, const std::vector<CallMat>* fuse_cm,
-                      cudaStream_t st) {
+                      int cautious, cudaStream_t st) {
   const Plan& P = h->plan;
   float* scale = reinterpret_cast<float*>(h->ws + P.off_scale);
   if (P.mode == MUON_MODE_FP32_VALIDATE) {
@@ -539,9 +558,11 @@ muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, const s
             TcApply& a = at.m[j];
             a.w = c.param;
             a.lrs = c.lrs;
+            a.lrwd = c.lrwd;
             a.flags = (uint16_t)((c.param_bf16 ? kApplyBf16 : 0) | (m.transposed ? kApplyTransposed : 0) |
-                                 (m.cols % 8 == 0 ? kApplyVec : 0));
+                                 (m.cols % 8 == 0 ? kApplyVec : 0) | (cautious ? kApplyCautious : 0));
             a.pad = 0;
+            a.pad2 = 0;
           }
           prof_begin(h, st);
           e = launch_tc_update_apply(*tp, at, clusters, st);
@@ -605,8 +626,10 @@ muon_status finish_call(muon_handle* h, cudaStream_t st) {
 }
 
 muon_status run(muon_handle* h, const std::vector<CallMat>& cm, const int64_t* rows, const int64_t* cols,
-                bool step, float mu, int nesterov, const float* coeffs, int ns_steps, float eps,
-                muon_mode mode, cudaStream_t st) {
+                bool step, const CallOpts& o, cudaStream_t st) {
+  const float* coeffs = o.coeffs;
+  const int ns_steps = o.ns_steps;
+  const muon_mode mode = o.mode;
   const int n = (int)cm.size();
   DeviceGuard dg(h->device);
   if (!dg.ok) return fail(h, MUON_ERR_CUDA, "cannot select device %d", h->device);
@@ -629,10 +652,9 @@ muon_status run(muon_handle* h, const std::vector<CallMat>& cm, const int64_t* r
     h->apply_table = new (std::nothrow) TcApplyTable();
     if (!h->apply_table) return fail(h, MUON_ERR_OOM, "host allocation of the weight-update table failed");
   }
-  if ((s = launch_elementwise(h, cm, true, 0, 0, mu, nesterov, eps, st))) return s;
-  if ((s = launch_ns(h, coeffs, ns_steps, fuse ? &cm : nullptr, st))) return s;
-  if (!fuse && (s = launch_elementwise(h, cm, false, step ? kEwApply : kEwExport, final_buf, mu, nesterov, eps, st)))
-    return s;
+  if ((s = launch_elementwise(h, cm, true, 0, 0, o, st))) return s;
+  if ((s = launch_ns(h, coeffs, ns_steps, fuse ? &cm : nullptr, o.cautious, st))) return s;
+  if (!fuse && (s = launch_elementwise(h, cm, false, step ? kEwApply : kEwExport, final_buf, o, st))) return s;
   return finish_call(h, st);
 }
 
@@ -666,10 +688,17 @@ muon_status muon_init(muon_handle_t* out, int device) {
   return MUON_OK;
 }
 
-muon_status muon_step(muon_handle_t h, const muon_matrix* mats, int n, float lr, float momentum, int nesterov,
-                      const float* coeffs, int ns_steps, float eps, muon_mode mode, void* cuda_stream) {
+}  // extern "C"
+
+namespace {
+
+muon_status step_impl(muon_handle_t h, const muon_matrix* mats, int n, float lr, float momentum, int nesterov,
+                      int lerp, const float* coeffs, int ns_steps, float eps, muon_mode mode, float weight_decay,
+                      int cautious, void* cuda_stream) {
   if (!h) return MUON_ERR_INVALID_ARG;
   h->err.clear();
+  if (!finite(weight_decay) || weight_decay < 0.f)
+    return fail(h, MUON_ERR_INVALID_ARG, "weight_decay must be finite and >= 0");
   if (n < 0 || n > kMaxMatrices) return fail(h, MUON_ERR_INVALID_ARG, "n = %d outside 0..%d", n, kMaxMatrices);
   if (n == 0) return MUON_OK;
   if (!mats) return fail(h, MUON_ERR_INVALID_ARG, "mats is NULL");
@@ -706,11 +735,38 @@ muon_status muon_step(muon_handle_t h, const muon_matrix* mats, int n, float lr,
     cols[i] = m.cols;
     const double scale = std::sqrt(std::max(1.0, (double)m.rows / (double)m.cols));
     cm[i] = CallMat{m.param, m.grad, m.momentum, nullptr, m.param_dtype == MUON_BF16, m.grad_dtype == MUON_BF16,
-                    (float)((double)lr * scale)};
+                    (float)((double)lr * scale), (float)((double)lr * (double)weight_decay)};
   }
   if ((s = check_overlaps(h, ranges))) return s;
-  return run(h, cm, rows.data(), cols.data(), true, momentum, nesterov ? 1 : 0, coeffs, ns_steps, eps, mode,
-             static_cast<cudaStream_t>(cuda_stream));
+  CallOpts o;
+  o.mu = momentum;
+  o.nesterov = nesterov ? 1 : 0;
+  o.lerp = lerp ? 1 : 0;
+  o.cautious = cautious ? 1 : 0;
+  o.coeffs = coeffs;
+  o.ns_steps = ns_steps;
+  o.eps = eps;
+  o.mode = mode;
+  return run(h, cm, rows.data(), cols.data(), true, o, static_cast<cudaStream_t>(cuda_stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+muon_status muon_step(muon_handle_t h, const muon_matrix* mats, int n, float lr, float momentum, int nesterov,
+                      const float* coeffs, int ns_steps, float eps, muon_mode mode, void* cuda_stream) {
+  return step_impl(h, mats, n, lr, momentum, nesterov, 0, coeffs, ns_steps, eps, mode, 0.f, 0, cuda_stream);
+}
+
+muon_status muon_step_ex(muon_handle_t h, const muon_matrix* mats, int n, const muon_options* opt,
+                         void* cuda_stream) {
+  if (!h) return MUON_ERR_INVALID_ARG;
+  if (!opt) return fail(h, MUON_ERR_INVALID_ARG, "options pointer is NULL");
+  if (opt->momentum_form != MUON_MOMENTUM_SGD && opt->momentum_form != MUON_MOMENTUM_LERP)
+    return fail(h, MUON_ERR_INVALID_ARG, "unknown momentum form %d", (int)opt->momentum_form);
+  return step_impl(h, mats, n, opt->lr, opt->momentum, opt->nesterov, opt->momentum_form == MUON_MOMENTUM_LERP,
+                   opt->coeffs, opt->ns_steps, opt->eps, opt->mode, opt->weight_decay, opt->cautious, cuda_stream);
 }
 
 muon_status muon_newton_schulz(muon_handle_t h, const void* const* x_in, void* const* o_out, const int64_t* rows,
@@ -739,7 +795,7 @@ muon_status muon_newton_schulz(muon_handle_t h, const void* const* x_in, void* c
       return fail(h, MUON_ERR_INVALID_ARG, "matrix %d has a pointer that is not 16-byte aligned", i);
     const size_t bytes = (size_t)rows[i] * (size_t)cols[i] * esz;
     ranges.push_back({(uintptr_t)o_out[i], (uintptr_t)o_out[i] + bytes, i});
-    cm[i] = CallMat{const_cast<void*>(x_in[i]), nullptr, nullptr, o_out[i], dtype == MUON_BF16, false, 0.f};
+    cm[i] = CallMat{const_cast<void*>(x_in[i]), nullptr, nullptr, o_out[i], dtype == MUON_BF16, false, 0.f, 0.f};
   }
   if ((s = check_overlaps(h, ranges))) return s;
   // outputs must not overlap any input either
@@ -749,7 +805,12 @@ muon_status muon_newton_schulz(muon_handle_t h, const void* const* x_in, void* c
       if (lo < r.hi && r.lo < hi)
         return fail(h, MUON_ERR_INVALID_ARG, "output of matrix %d overlaps input of matrix %d", r.mat, i);
   }
-  return run(h, cm, rows, cols, false, 0.f, 0, coeffs, ns_steps, eps, mode, static_cast<cudaStream_t>(cuda_stream));
+  CallOpts o;
+  o.coeffs = coeffs;
+  o.ns_steps = ns_steps;
+  o.eps = eps;
+  o.mode = mode;
+  return run(h, cm, rows, cols, false, o, static_cast<cudaStream_t>(cuda_stream));
 }
 
 muon_status muon_selftest_wait_timeout(muon_handle_t h, int64_t limit_ns, void* cuda_stream) {

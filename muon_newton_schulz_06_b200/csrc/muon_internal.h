@@ -41,6 +41,7 @@ struct EwMat {
   uint8_t param_bf16;   // dtype of `param` (apply / export / normalise input)
   uint8_t grad_bf16;    // dtype of `grad`
   float lrs;            // fl32(lr * sqrt(max(1, rows/cols))) (apply)
+  float lrwd;           // fl32(lr * weight_decay) (apply; 0 = no decay)
 };
 
 struct EwParams {
@@ -50,6 +51,9 @@ struct EwParams {
   float mu;
   int nesterov;
   int use_momentum;     // 0: U = x_in (Newton-Schulz entry point)
+  int lerp;             // interpolation-form momentum
+  float omu;            // fl32(1 - mu)
+  int cautious;         // decay only where O * W >= 0
   float eps;
   float* partials;      // per (unit, warp) sum of squares
   float* scale;         // per-matrix 1/(||U||_F + eps)
@@ -114,13 +118,15 @@ struct __align__(64) TcParams {
 
 // Weight update fused into the last Update pass: W <- RNE(fl32(W - fl32(lrs * O))) with
 // O = bf16(X_K), exactly what the separate apply pass computes; X_K itself is not stored.
-constexpr int kMaxFusedApply = 1024;
-enum : uint16_t { kApplyBf16 = 1, kApplyTransposed = 2, kApplyVec = 4 };
+constexpr int kMaxFusedApply = 768;
+enum : uint16_t { kApplyBf16 = 1, kApplyTransposed = 2, kApplyVec = 4, kApplyCautious = 8 };
 struct TcApply {
   void* w;         // caller weight, rows x cols row-major
   float lrs;       // fl32(lr * sqrt(max(1, rows/cols)))
-  uint16_t flags;  // kApplyBf16 | kApplyTransposed (rows > cols) | kApplyVec (16-byte rows)
+  float lrwd;      // fl32(lr * weight_decay), 0 = no decay
+  uint16_t flags;  // kApplyBf16 | kApplyTransposed (rows > cols) | kApplyVec (16-byte rows) | kApplyCautious
   uint16_t pad;
+  uint32_t pad2;
 };
 struct __align__(16) TcApplyTable {
   int base;        // global index of entry 0

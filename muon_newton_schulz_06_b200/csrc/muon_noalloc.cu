@@ -145,6 +145,8 @@ extern "C" MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, voi
   g_ew.n_mats = 1;
   g_ew.total_units = n_units;
   g_ew.use_momentum = 0;
+  g_ew.lerp = 0;
+  g_ew.cautious = 0;
   g_ew.eps = eps;
   g_ew.partials = reinterpret_cast<float*>(scr + off_part);
   g_ew.scale = reinterpret_cast<float*>(scr + off_scale);

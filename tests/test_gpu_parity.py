@@ -214,7 +214,7 @@ def test_grouped_step_matches_single_matrix_calls(mb, handle):
 
 
 def test_fused_and_separate_apply_agree(mb, handle):
-    """More matrices than one fused weight-update table holds (1024) take the separate
+    """More matrices than one fused weight-update table holds (768) take the separate
     apply pass; the same matrices in two smaller calls take the fused epilogue.  Both
     must give the same bits."""
     n = 1100
