@@ -32,4 +32,5 @@ from .muon import (  # noqa: F401
     muon_step_matrix,
     muon_step,
     cautious_mask,
+    normuon_rescale,
 )

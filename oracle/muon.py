@@ -35,6 +35,7 @@ design notes of the library):
   (g x parameter) >= 0, read with g = O, the update that is applied).
 * The interpolation form of the momentum (M <- mu*M + (1-mu)*G) is an option next to
   the default SGD form.
+* NorMuon is optional (see ``normuon_rescale`` for its readings).
 """
 from __future__ import annotations
 
@@ -123,14 +124,40 @@ def cautious_mask(o, w):
     return (np.asarray(o, dtype=np.float64) * np.asarray(w, dtype=np.float64)) >= 0
 
 
+def normuon_rescale(o, v, beta2: float, eps: float):
+    """NorMuon (autoresearch review, MuonAdamW paragraph): after orthogonalisation, a
+    second-moment estimate per row -- or per column, by aspect ratio -- kept as an EMA
+    and used to give every output dimension its own step size.
+
+    Readings: the statistics run over the longer dimension, one per index of the
+    shorter one (rows of a wide matrix, columns of a tall one); v <- beta2*v +
+    (1-beta2)*mean(O^2); O' = O / (sqrt(v) + eps); O' is rescaled to the Frobenius norm
+    of O, which keeps the step size's meaning and makes a bias correction of v
+    unnecessary (it would scale every row alike).  Returns (O'' float64, v_new float64).
+    """
+    o = np.asarray(o, dtype=np.float64)
+    rows, cols = o.shape
+    per_row = rows <= cols
+    q = np.mean(o * o, axis=1 if per_row else 0)
+    v_new = beta2 * np.asarray(v, dtype=np.float64) + (1.0 - beta2) * q
+    f = 1.0 / (np.sqrt(v_new) + eps)
+    o1 = o * (f[:, None] if per_row else f[None, :])
+    n0, n1 = math.sqrt(float(np.sum(o * o))), math.sqrt(float(np.sum(o1 * o1)))
+    o2 = o1 * (n0 / n1) if n1 > 0 else o1
+    return o2, v_new
+
+
 def muon_step_matrix(w, grad, momentum, *, lr: float, mu: float, nesterov: bool = True,
                      coeffs: Sequence[Sequence[float]] | None = None, eps: float = 1e-7,
-                     lerp: bool = False, weight_decay: float = 0.0, cautious: bool = False):
+                     lerp: bool = False, weight_decay: float = 0.0, cautious: bool = False,
+                     normuon_state=None, normuon_beta2: float = 0.95, normuon_eps: float = 1e-8):
     """One Muon step for one matrix.
 
     Returns (W_new float64, M_new float32, O float64).  W_new is the exact
     W - lr*scale*O - lr*weight_decay*mask*W with mask = 1 everywhere, or the cautious
     mask when ``cautious``; rounding to the parameter's dtype is the caller's concern.
+    With ``normuon_state`` (the previous second-moment vector), O is replaced by its
+    NorMuon rescaling and the function returns (W_new, M_new, O'', v_new).
     """
     if coeffs is None:
         coeffs = [QUINTIC] * 5
@@ -139,10 +166,15 @@ def muon_step_matrix(w, grad, momentum, *, lr: float, mu: float, nesterov: bool 
     m_new, u = nesterov_momentum_f32(grad, momentum, mu, nesterov, lerp=lerp)
     x0 = frobenius_normalise(u, eps)
     o = newton_schulz(x0, coeffs)
+    v_new = None
+    if normuon_state is not None:
+        o, v_new = normuon_rescale(o, normuon_state, normuon_beta2, normuon_eps)
     w_new = w64 - lr * update_scale(rows, cols) * o
     if weight_decay:
         mask = cautious_mask(o, w64) if cautious else np.ones_like(w64, dtype=bool)
         w_new = w_new - lr * weight_decay * np.where(mask, w64, 0.0)
+    if v_new is not None:
+        return w_new, m_new, o, v_new
     return w_new, m_new, o
 
 

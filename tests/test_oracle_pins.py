@@ -345,3 +345,39 @@ def test_weight_decay_and_cautious_mask_closed_form():
     assert np.allclose(w_cwd, w - 0.1 * np.diag(od) - 0.05 * np.where(mask, w, 0.0), atol=1e-15)
     w_wd, _, _ = oracle.muon_step_matrix(w, g, z, lr=0.1, mu=0.0, coeffs=coeffs, eps=0.0, weight_decay=0.5)
     assert np.allclose(w_wd, w_plain - 0.05 * w, atol=1e-15)
+
+
+# ---------------------------------------------------------------- NorMuon
+
+@pytest.mark.parametrize("rows,cols", [(3, 5), (5, 3), (4, 4)])
+def test_normuon_on_a_diagonal_input(rows, cols):
+    """Diagonal O (entries d_i): one statistic per index of the shorter dimension,
+    q_i = d_i^2 / L; from v = 0, v = (1-b2) q, so O' = d_i / (sqrt(1-b2) d_i/sqrt(L) + eps)
+    is (nearly) the same for every i, and O'' has O's Frobenius norm."""
+    k = min(rows, cols)
+    L = max(rows, cols)
+    d = np.array([0.9, 0.5, 0.25, 0.1][:k])
+    o = np.zeros((rows, cols))
+    o[np.arange(k), np.arange(k)] = d
+    o2, v = oracle.normuon_rescale(o, np.zeros(k), 0.9, 1e-12)
+    assert np.allclose(v, 0.1 * d ** 2 / L, rtol=1e-14)
+    diag = o2[np.arange(k), np.arange(k)]
+    assert np.allclose(diag, diag[0], rtol=1e-9)
+    assert np.isclose(np.linalg.norm(o2), np.linalg.norm(o), rtol=1e-14)
+    assert np.count_nonzero(o2) == k
+    # second step with the same O: v = 0.9 v1 + 0.1 q = 0.19 q
+    _, v2 = oracle.normuon_rescale(o, v, 0.9, 1e-12)
+    assert np.allclose(v2, 0.19 * d ** 2 / L, rtol=1e-13)
+
+
+def test_normuon_rows_vs_columns_by_aspect():
+    rng = np.random.default_rng(77)
+    o = rng.standard_normal((4, 9))
+    _, v_wide = oracle.normuon_rescale(o, np.zeros(4), 0.0, 0.0)
+    assert np.allclose(v_wide, np.mean(o ** 2, axis=1))
+    _, v_tall = oracle.normuon_rescale(o.T, np.zeros(4), 0.0, 0.0)
+    assert np.allclose(v_tall, np.mean(o ** 2, axis=1))
+    # transposing the input transposes the output
+    a, _ = oracle.normuon_rescale(o, np.full(4, 0.3), 0.5, 1e-6)
+    b, _ = oracle.normuon_rescale(o.T, np.full(4, 0.3), 0.5, 1e-6)
+    assert np.allclose(a, b.T, rtol=1e-14)
