@@ -138,6 +138,21 @@ typedef struct {
   muon_mode mode;
   float weight_decay;
   int cautious;
+  /* NorMuon (autoresearch train.py review, MuonAdamW paragraph: a per-row -- or, by
+   * aspect ratio, per-column -- second moment of the orthogonalised update, kept as an
+   * EMA, scales the update per output dimension).  With s = min(rows, cols),
+   * L = max(rows, cols) and i running over the shorter dimension:
+   *   q_i = sum over the longer dimension of O_i^2 / L          (fp32 sums)
+   *   v_i <- fl32(fl32(beta2*v_i) + fl32((1-beta2)*q_i))
+   *   f_i = 1/(sqrt(v_i) + eps),  r = sqrt(sum_i q_i / sum_i q_i f_i^2)
+   *   O  <- fl32(fl32(f_i*r) * O)                               (same Frobenius norm)
+   * before the update (and the cautious mask) use O.  normuon_state is a HOST array of
+   * n DEVICE pointers, each to s float32 values (16-byte aligned, zero before the
+   * first step), updated in place.  The weight update then runs as a separate pass. */
+  int normuon;
+  float normuon_beta2;          /* [0, 1) */
+  float normuon_eps;            /* > 0 */
+  float* const* normuon_state;
 } muon_options;
 
 /* muon_step with every option; `opt` is a HOST pointer.  muon_step(h, mats, n, lr, mu,

@@ -62,7 +62,9 @@ class muon_options(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_float), ("momentum", ctypes.c_float), ("nesterov", ctypes.c_int),
                 ("momentum_form", ctypes.c_int), ("coeffs", ctypes.POINTER(ctypes.c_float)),
                 ("ns_steps", ctypes.c_int), ("eps", ctypes.c_float), ("mode", ctypes.c_int),
-                ("weight_decay", ctypes.c_float), ("cautious", ctypes.c_int)]
+                ("weight_decay", ctypes.c_float), ("cautious", ctypes.c_int),
+                ("normuon", ctypes.c_int), ("normuon_beta2", ctypes.c_float), ("normuon_eps", ctypes.c_float),
+                ("normuon_state", ctypes.POINTER(ctypes.c_void_p))]
 
 
 _lib_handle = None
@@ -201,17 +203,33 @@ def muon_step(handle, params: Sequence[torch.Tensor], grads: Sequence[torch.Tens
 def muon_step_ex(handle, params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor],
                  moms: Sequence[torch.Tensor], lr: float, momentum: float = 0.95, nesterov: bool = True,
                  momentum_form: str = "sgd", coeffs=None, ns_steps: int = 5, eps: float = 1e-7, mode="bf16",
-                 weight_decay: float = 0.0, cautious: bool = False, stream=None) -> None:
+                 weight_decay: float = 0.0, cautious: bool = False, normuon_state=None,
+                 normuon_beta2: float = 0.95, normuon_eps: float = 1e-8, stream=None) -> None:
     """muon_step with every option: momentum_form "sgd" or "lerp"; weight_decay (0 = off);
-    cautious (decay only where the update and the weight agree in sign)."""
+    cautious (decay only where the update and the weight agree in sign); normuon_state
+    (list of float32 CUDA vectors of min(rows, cols) entries, zero at the start) turns
+    on the NorMuon rescaling and is updated in place."""
     forms = {"sgd": MUON_MOMENTUM_SGD, "lerp": MUON_MOMENTUM_LERP}
     if momentum_form not in forms:
         raise ValueError(f"unknown momentum_form {momentum_form!r}")
     arr, n = _matrix_array(params, grads, moms)
     dev = params[0].device if n else torch.device("cuda")
     c = _coeff_array(coeffs, ns_steps)
+    ns_arr = None
+    if normuon_state is not None:
+        if len(normuon_state) != n:
+            raise ValueError("normuon_state must hold one vector per matrix")
+        ns_arr = (ctypes.c_void_p * max(n, 1))()
+        for i, (v, w) in enumerate(zip(normuon_state, params)):
+            if not (isinstance(v, torch.Tensor) and v.is_cuda and v.dtype == torch.float32 and v.is_contiguous()):
+                raise TypeError("normuon_state entries must be contiguous float32 CUDA tensors")
+            if v.numel() != min(w.shape):
+                raise ValueError(f"normuon_state[{i}] must have min(rows, cols) = {min(w.shape)} entries")
+            ns_arr[i] = v.data_ptr()
     opt = muon_options(float(lr), float(momentum), 1 if nesterov else 0, forms[momentum_form], c, int(ns_steps),
-                       float(eps), _mode_code(mode), float(weight_decay), 1 if cautious else 0)
+                       float(eps), _mode_code(mode), float(weight_decay), 1 if cautious else 0,
+                       1 if normuon_state is not None else 0, float(normuon_beta2), float(normuon_eps),
+                       ns_arr)
     _check(load_library().muon_step_ex(handle, arr, n, ctypes.byref(opt), _stream_ptr(stream, dev)), handle)
 
 

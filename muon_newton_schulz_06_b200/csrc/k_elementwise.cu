@@ -231,6 +231,93 @@ norm_finalize_kernel(const __grid_constant__ EwParams p) {
   }
 }
 
+// NorMuon statistics: one warp per row of the wide orientation (s rows of length L):
+// q = sum of O^2 / L in a fixed order (lane stride, then a shuffle tree); the caller's
+// state v is updated in place; rowsq keeps the sum, rowf the factor 1/(sqrt(v)+eps).
+template <typename WT>
+__global__ void __launch_bounds__(kThreads)
+normuon_rows_kernel(const __grid_constant__ EwParams p, int row_end) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * kThreads + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * kThreads) >> 5;
+  for (int grow = p.mats[0].row_base + gw; grow < row_end; grow += nw) {
+    int lo = 0, hi = p.n_mats - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.mats[mid].row_base <= grow) lo = mid; else hi = mid - 1;
+    }
+    const EwMat& m = p.mats[lo];
+    const int i = grow - m.row_base;
+    const int L = m.transposed ? m.rows : m.cols;
+    const WT* x = reinterpret_cast<const WT*>(m.work) + (size_t)i * m.ld;
+    float acc = 0.f;
+    for (int l = 8 * lane; l < L; l += 256) {
+      float v[8];
+      if (l + 8 <= L) {
+        ld8(x, l, sizeof(WT) == 2, v);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float t = 0.f;
+          if (l + q < L) {
+            if constexpr (sizeof(WT) == 2) t = __bfloat162float(x[l + q]);
+            else t = x[l + q];
+          }
+          v[q] = t;
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc = fmaf(v[q], v[q], acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      const float q = __fdiv_rn(acc, (float)L);
+      const float vn = __fadd_rn(__fmul_rn(p.nb2, m.nstate[i]), __fmul_rn(__fsub_rn(1.f, p.nb2), q));
+      m.nstate[i] = vn;
+      p.rowsq[grow] = acc;
+      p.rowf[grow] = 1.f / (sqrtf(vn) + p.neps);
+    }
+  }
+}
+
+// Per matrix: r = sqrt(sum q_i / sum q_i f_i^2) in double, fixed order; then
+// rowsq[i] <- fl32(f_i * r), the factor the apply pass multiplies O by.
+__global__ void __launch_bounds__(kThreads)
+normuon_matrix_kernel(const __grid_constant__ EwParams p) {
+  __shared__ double red[2][kThreads / 32];
+  __shared__ float rr;
+  const EwMat& m = p.mats[blockIdx.x];
+  const int s = m.transposed ? m.cols : m.rows;
+  double a = 0.0, b = 0.0;
+  for (int i = threadIdx.x; i < s; i += kThreads) {
+    const double q = p.rowsq[m.row_base + i], f = p.rowf[m.row_base + i];
+    a += q;
+    b += q * f * f;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    red[0][threadIdx.x >> 5] = a;
+    red[1][threadIdx.x >> 5] = b;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double ta = 0.0, tb = 0.0;
+    for (int w = 0; w < kThreads / 32; ++w) {
+      ta += red[0][w];
+      tb += red[1][w];
+    }
+    rr = (tb > 0.0) ? (float)sqrt(ta / tb) : 1.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < s; i += kThreads)
+    p.rowsq[m.row_base + i] = __fmul_rn(p.rowf[m.row_base + i], rr);
+}
+
 template <typename WT>
 __global__ void __launch_bounds__(kThreads)
 apply_kernel(const __grid_constant__ EwParams p, int out_kind) {
@@ -305,6 +392,14 @@ apply_kernel(const __grid_constant__ EwParams p, int out_kind) {
       if (r >= m.rows) continue;
       const bool full = c + 8 <= m.cols;
       const size_t base = (size_t)r * m.cols + c;
+      if (p.normuon) {
+        // per-row factor of the wide orientation: caller row (wide) or column (tall)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int wi = m.transposed ? (c + q < m.cols ? c + q : 0) : r;
+          o[pr][q] = __fmul_rn(p.rowsq[m.row_base + wi], o[pr][q]);
+        }
+      }
       if (out_kind == kEwApply) {
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -338,6 +433,18 @@ cudaError_t launch_momentum_norm(const EwParams& p, bool work_f32, int grid, cud
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   norm_finalize_kernel<<<p.n_mats, kThreads, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_normuon(const EwParams& p, bool work_f32, int grid, cudaStream_t st) {
+  if (p.n_mats == 0) return cudaSuccess;
+  const EwMat& last = p.mats[p.n_mats - 1];
+  const int row_end = last.row_base + (last.transposed ? last.cols : last.rows);
+  if (work_f32) normuon_rows_kernel<float><<<grid, kThreads, 0, st>>>(p, row_end);
+  else normuon_rows_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(p, row_end);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  normuon_matrix_kernel<<<p.n_mats, kThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 

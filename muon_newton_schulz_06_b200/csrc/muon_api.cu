@@ -46,6 +46,7 @@ struct GroupPlan {
 
 struct MatPlan {
   int group = 0, idx = 0, gid = 0;
+  int row_base = 0;  // first entry in the NorMuon row arrays (prefix of min(rows, cols))
   int64_t rows = 0, cols = 0;
   bool transposed = false;
   int n_units = 0, part_base = 0, tiles_c = 0;
@@ -66,7 +67,8 @@ struct Plan {
   std::vector<int> mat_of_gid;  // caller index of each global (group-major) index
   std::vector<ChunkPlan> chunks;
   std::vector<TcTile> tiles;  // host copy of every chunk's tile lists
-  size_t off_partials = 0, off_scale = 0, off_tiles = 0, bytes = 0;
+  size_t off_partials = 0, off_scale = 0, off_tiles = 0, off_rowsq = 0, off_rowf = 0, bytes = 0;
+  int total_rows = 0;
   int total_units = 0;
   // TMA maps per group (bf16 mode): X K-major (ping/pong), X MN-major (ping/pong), Gram, Poly
   std::vector<CUtensorMap> map_xk[2], map_xmn[2], map_gram, map_poly;
@@ -247,6 +249,8 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
     m.n_units = (int)((rows[i] + kEwTile - 1) / kEwTile) * m.tiles_c;
     m.part_base = P.total_units;
     P.total_units += m.n_units;
+    m.row_base = P.total_rows;
+    P.total_rows += s;
   }
   // global matrix index = group-major order
   int gid = 0;
@@ -271,6 +275,8 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
   }
   P.off_partials = off; off = align_up(off + (size_t)P.total_units * kWarpsPerUnit * 4, 256);
   P.off_scale = off; off = align_up(off + (size_t)n * 4, 256);
+  P.off_rowsq = off; off = align_up(off + (size_t)P.total_rows * 4, 256);
+  P.off_rowf = off; off = align_up(off + (size_t)P.total_rows * 4, 256);
   // tile lists (tensor-core path)
   if (mode == MUON_MODE_BF16) {
     for (int g0 = 0; g0 < (int)P.groups.size(); g0 += kMaxGroups) {
@@ -381,6 +387,7 @@ struct CallMat {
   bool param_bf16, grad_bf16;
   float lrs;          // fl32(lr * sqrt(max(1, rows/cols)))
   float lrwd;         // fl32(lr * weight_decay)
+  float* nstate;      // NorMuon second moments (device, min(rows, cols) floats) or null
 };
 
 // Per-call options shared by every matrix.
@@ -393,7 +400,11 @@ struct CallOpts {
   int ns_steps = 5;
   float eps = 0.f;
   muon_mode mode = MUON_MODE_BF16;
+  int normuon = 0;
+  float nb2 = 0.f, neps = 0.f;
 };
+
+enum EwPass { kPassMomentum = 0, kPassOut = 1, kPassNormuon = 2 };
 
 void* work_ptr(muon_handle* h, const MatPlan& m, int buf) {
   const Plan& P = h->plan;
@@ -402,8 +413,9 @@ void* work_ptr(muon_handle* h, const MatPlan& m, int buf) {
   return h->ws + g.off_x[buf] + (size_t)m.idx * g.s * g.ld_x * esz;
 }
 
-muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, bool momentum_pass,
-                               int out_kind, int work_buf, const CallOpts& o, cudaStream_t st) {
+muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, int pass, int out_kind,
+                               int work_buf, const CallOpts& o, cudaStream_t st) {
+  const bool momentum_pass = pass == kPassMomentum;
   const float mu = o.mu, eps = o.eps;
   const int nesterov = o.nesterov;
   const Plan& P = h->plan;
@@ -419,6 +431,11 @@ muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, b
     ep->lerp = o.lerp;
     ep->omu = 1.0f - mu;
     ep->cautious = o.cautious;
+    ep->normuon = (pass == kPassOut && o.normuon) ? 1 : 0;
+    ep->nb2 = o.nb2;
+    ep->neps = o.neps;
+    ep->rowsq = reinterpret_cast<float*>(h->ws + P.off_rowsq);
+    ep->rowf = reinterpret_cast<float*>(h->ws + P.off_rowf);
     ep->eps = eps;
     ep->partials = reinterpret_cast<float*>(h->ws + P.off_partials);
     ep->scale = reinterpret_cast<float*>(h->ws + P.off_scale);
@@ -447,17 +464,22 @@ muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, b
       e.grad_bf16 = cm[i].grad_bf16 ? 1 : 0;
       e.lrs = cm[i].lrs;
       e.lrwd = cm[i].lrwd;
+      e.nstate = cm[i].nstate;
+      e.row_base = m.row_base;
       units += m.n_units;
     }
     ep->total_units = units;
     const int grid = std::max(1, std::min(units, h->sm_count * 8));
     prof_begin(h, st);
-    cudaError_t err = momentum_pass ? launch_momentum_norm(*ep, f32, grid, st)
-                                    : launch_apply(*ep, f32, out_kind, grid, st);
-    prof_end(h, momentum_pass ? MUON_KIND_MOMENTUM_NORM : MUON_KIND_APPLY, st);
+    cudaError_t err = pass == kPassMomentum ? launch_momentum_norm(*ep, f32, grid, st)
+                      : pass == kPassNormuon ? launch_normuon(*ep, f32, h->sm_count * 8, st)
+                                             : launch_apply(*ep, f32, out_kind, grid, st);
+    prof_end(h, pass == kPassMomentum ? MUON_KIND_MOMENTUM_NORM : MUON_KIND_APPLY, st);
     delete ep;
-    if (err != cudaSuccess) return cuda_fail(h, err, momentum_pass ? "momentum/norm launch" : "apply launch");
-    h->last_launches += momentum_pass ? 2 : 1;
+    if (err != cudaSuccess)
+      return cuda_fail(h, err, pass == kPassMomentum ? "momentum/norm launch"
+                               : pass == kPassNormuon ? "NorMuon launch" : "apply launch");
+    h->last_launches += pass == kPassOut ? 1 : 2;
   }
   return MUON_OK;
 }
@@ -647,14 +669,15 @@ muon_status run(muon_handle* h, const std::vector<CallMat>& cm, const int64_t* r
     if ((s = build_plan(h, rows, cols, n, mode, st))) return s;
   }
   const int final_buf = ns_steps & 1;
-  const bool fuse = step && can_fuse_apply(h->plan);
+  const bool fuse = step && !o.normuon && can_fuse_apply(h->plan);
   if (fuse && !h->apply_table) {
     h->apply_table = new (std::nothrow) TcApplyTable();
     if (!h->apply_table) return fail(h, MUON_ERR_OOM, "host allocation of the weight-update table failed");
   }
-  if ((s = launch_elementwise(h, cm, true, 0, 0, o, st))) return s;
+  if ((s = launch_elementwise(h, cm, kPassMomentum, 0, 0, o, st))) return s;
   if ((s = launch_ns(h, coeffs, ns_steps, fuse ? &cm : nullptr, o.cautious, st))) return s;
-  if (!fuse && (s = launch_elementwise(h, cm, false, step ? kEwApply : kEwExport, final_buf, o, st))) return s;
+  if (step && o.normuon && (s = launch_elementwise(h, cm, kPassNormuon, 0, final_buf, o, st))) return s;
+  if (!fuse && (s = launch_elementwise(h, cm, kPassOut, step ? kEwApply : kEwExport, final_buf, o, st))) return s;
   return finish_call(h, st);
 }
 
@@ -694,11 +717,17 @@ namespace {
 
 muon_status step_impl(muon_handle_t h, const muon_matrix* mats, int n, float lr, float momentum, int nesterov,
                       int lerp, const float* coeffs, int ns_steps, float eps, muon_mode mode, float weight_decay,
-                      int cautious, void* cuda_stream) {
+                      int cautious, int normuon, float nb2, float neps, float* const* nstate, void* cuda_stream) {
   if (!h) return MUON_ERR_INVALID_ARG;
   h->err.clear();
   if (!finite(weight_decay) || weight_decay < 0.f)
     return fail(h, MUON_ERR_INVALID_ARG, "weight_decay must be finite and >= 0");
+  if (normuon) {
+    if (!finite(nb2) || nb2 < 0.f || nb2 >= 1.f)
+      return fail(h, MUON_ERR_INVALID_ARG, "normuon_beta2 must lie in [0, 1)");
+    if (!finite(neps) || neps <= 0.f) return fail(h, MUON_ERR_INVALID_ARG, "normuon_eps must be finite and > 0");
+    if (n > 0 && !nstate) return fail(h, MUON_ERR_INVALID_ARG, "normuon_state is NULL");
+  }
   if (n < 0 || n > kMaxMatrices) return fail(h, MUON_ERR_INVALID_ARG, "n = %d outside 0..%d", n, kMaxMatrices);
   if (n == 0) return MUON_OK;
   if (!mats) return fail(h, MUON_ERR_INVALID_ARG, "mats is NULL");
@@ -734,8 +763,16 @@ muon_status step_impl(muon_handle_t h, const muon_matrix* mats, int n, float lr,
     rows[i] = m.rows;
     cols[i] = m.cols;
     const double scale = std::sqrt(std::max(1.0, (double)m.rows / (double)m.cols));
+    float* ns_ptr = nullptr;
+    if (normuon) {
+      ns_ptr = nstate[i];
+      if (!ns_ptr || (reinterpret_cast<uintptr_t>(ns_ptr) & 15u))
+        return fail(h, MUON_ERR_INVALID_ARG, "normuon_state[%d] is NULL or not 16-byte aligned", i);
+      const size_t sb = (size_t)std::min(m.rows, m.cols) * 4;
+      ranges.push_back({(uintptr_t)ns_ptr, (uintptr_t)ns_ptr + sb, i});
+    }
     cm[i] = CallMat{m.param, m.grad, m.momentum, nullptr, m.param_dtype == MUON_BF16, m.grad_dtype == MUON_BF16,
-                    (float)((double)lr * scale), (float)((double)lr * (double)weight_decay)};
+                    (float)((double)lr * scale), (float)((double)lr * (double)weight_decay), ns_ptr};
   }
   if ((s = check_overlaps(h, ranges))) return s;
   CallOpts o;
@@ -747,6 +784,9 @@ muon_status step_impl(muon_handle_t h, const muon_matrix* mats, int n, float lr,
   o.ns_steps = ns_steps;
   o.eps = eps;
   o.mode = mode;
+  o.normuon = normuon ? 1 : 0;
+  o.nb2 = nb2;
+  o.neps = neps;
   return run(h, cm, rows.data(), cols.data(), true, o, static_cast<cudaStream_t>(cuda_stream));
 }
 
@@ -756,7 +796,8 @@ extern "C" {
 
 muon_status muon_step(muon_handle_t h, const muon_matrix* mats, int n, float lr, float momentum, int nesterov,
                       const float* coeffs, int ns_steps, float eps, muon_mode mode, void* cuda_stream) {
-  return step_impl(h, mats, n, lr, momentum, nesterov, 0, coeffs, ns_steps, eps, mode, 0.f, 0, cuda_stream);
+  return step_impl(h, mats, n, lr, momentum, nesterov, 0, coeffs, ns_steps, eps, mode, 0.f, 0, 0, 0.f, 0.f, nullptr,
+                   cuda_stream);
 }
 
 muon_status muon_step_ex(muon_handle_t h, const muon_matrix* mats, int n, const muon_options* opt,
@@ -766,7 +807,8 @@ muon_status muon_step_ex(muon_handle_t h, const muon_matrix* mats, int n, const 
   if (opt->momentum_form != MUON_MOMENTUM_SGD && opt->momentum_form != MUON_MOMENTUM_LERP)
     return fail(h, MUON_ERR_INVALID_ARG, "unknown momentum form %d", (int)opt->momentum_form);
   return step_impl(h, mats, n, opt->lr, opt->momentum, opt->nesterov, opt->momentum_form == MUON_MOMENTUM_LERP,
-                   opt->coeffs, opt->ns_steps, opt->eps, opt->mode, opt->weight_decay, opt->cautious, cuda_stream);
+                   opt->coeffs, opt->ns_steps, opt->eps, opt->mode, opt->weight_decay, opt->cautious, opt->normuon,
+                   opt->normuon_beta2, opt->normuon_eps, opt->normuon_state, cuda_stream);
 }
 
 muon_status muon_newton_schulz(muon_handle_t h, const void* const* x_in, void* const* o_out, const int64_t* rows,
@@ -795,7 +837,8 @@ muon_status muon_newton_schulz(muon_handle_t h, const void* const* x_in, void* c
       return fail(h, MUON_ERR_INVALID_ARG, "matrix %d has a pointer that is not 16-byte aligned", i);
     const size_t bytes = (size_t)rows[i] * (size_t)cols[i] * esz;
     ranges.push_back({(uintptr_t)o_out[i], (uintptr_t)o_out[i] + bytes, i});
-    cm[i] = CallMat{const_cast<void*>(x_in[i]), nullptr, nullptr, o_out[i], dtype == MUON_BF16, false, 0.f, 0.f};
+    cm[i] = CallMat{const_cast<void*>(x_in[i]), nullptr, nullptr, o_out[i], dtype == MUON_BF16, false, 0.f, 0.f,
+                    nullptr};
   }
   if ((s = check_overlaps(h, ranges))) return s;
   // outputs must not overlap any input either

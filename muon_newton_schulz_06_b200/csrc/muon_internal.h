@@ -42,6 +42,8 @@ struct EwMat {
   uint8_t grad_bf16;    // dtype of `grad`
   float lrs;            // fl32(lr * sqrt(max(1, rows/cols))) (apply)
   float lrwd;           // fl32(lr * weight_decay) (apply; 0 = no decay)
+  float* nstate;        // NorMuon second moments (s floats) or null
+  int32_t row_base;     // first entry of this matrix in the NorMuon row arrays
 };
 
 struct EwParams {
@@ -54,12 +56,20 @@ struct EwParams {
   int lerp;             // interpolation-form momentum
   float omu;            // fl32(1 - mu)
   int cautious;         // decay only where O * W >= 0
+  int normuon;          // apply: scale O by the per-row NorMuon factor
+  float nb2, neps;      // NorMuon beta2, eps
+  float* rowsq;         // NorMuon: per-row sum of O^2, then per-row factor f_i * r
+  float* rowf;          // NorMuon: per-row 1/(sqrt(v)+eps)
   float eps;
   float* partials;      // per (unit, warp) sum of squares
   float* scale;         // per-matrix 1/(||U||_F + eps)
 };
 
 enum EwOut : int { kEwApply = 0, kEwExport = 1 };
+
+// NorMuon passes (k_elementwise.cu): per-row statistics and state update, then the
+// per-matrix norm-preserving factor; the apply pass reads the factors.
+cudaError_t launch_normuon(const EwParams& p, bool work_f32, int grid, cudaStream_t st);
 
 // Launchers (k_elementwise.cu).  work_f32 selects the workspace element type.
 // launch_momentum_norm enqueues two kernels: the pass and the per-matrix norm finalize.

@@ -145,3 +145,45 @@ def test_bad_options_are_rejected(mb):
             mb.muon_step_ex(h, [w], [w.clone()], [w.clone()], lr=0.1, momentum_form="adam")
     finally:
         mb.muon_destroy(h)
+
+
+# ---------------------------------------------------------------- NorMuon
+
+def normuon_run(mb, data, states, steps, **kw):
+    """`steps` NorMuon steps with fp32 zero weights reset before each step and lr = 1, so
+    that W' = -scale*O'' exactly (scale in {1, 2}); returns O'' of the last step."""
+    specs = data["specs"]
+    scales = [math.sqrt(max(1.0, s.rows / s.cols)) for s in specs]
+    M = [m.clone() for m in data["M"]]
+    h = mb.muon_init(0)
+    try:
+        for _ in range(steps):
+            W = [torch.zeros(s.rows, s.cols, device="cuda") for s in specs]
+            mb.muon_step_ex(h, W, data["G"], M, lr=1.0, normuon_state=states, **kw)
+        torch.cuda.synchronize()
+        mb.muon_sync(h)
+    finally:
+        mb.muon_destroy(h)
+    return [(-w / sc) for w, sc in zip(W, scales)], M
+
+
+@pytest.mark.parametrize("mode,tol", [("bf16", BF16_TOL), ("fp32", 1e-4)])
+def test_normuon_two_steps_vs_oracle(mb, mode, tol):
+    if mode == "bf16":
+        data = synth.make_matrix_set(1, device="cuda", layers=[0])
+    else:
+        d0 = synth.make_matrix_set(0)
+        data = {k: ([x.cuda() for x in v] if k in ("W", "G", "M") else v) for k, v in d0.items()}
+    states = [torch.zeros(min(s.rows, s.cols), device="cuda") for s in data["specs"]]
+    O2, M = normuon_run(mb, data, states, 2, mode=mode, normuon_beta2=0.9, normuon_eps=1e-8)
+    for i, spec in enumerate(data["specs"]):
+        g = data["G"][i].float().cpu().numpy()
+        m = data["M"][i].cpu().numpy()
+        v = np.zeros(min(spec.rows, spec.cols))
+        for _ in range(2):
+            _, m, o2, v = oracle.muon_step_matrix(np.zeros((spec.rows, spec.cols)), g, m, lr=1.0, mu=0.95,
+                                                  normuon_state=v, normuon_beta2=0.9, normuon_eps=1e-8)
+        err = rel(O2[i].double().cpu().numpy(), o2)
+        assert err < tol, (spec, err)
+        vt = states[i].double().cpu().numpy()
+        assert rel(vt, v) < 2 * tol + 1e-6, (spec, rel(vt, v))
