@@ -56,6 +56,9 @@ def parse():
     ap.add_argument("--shard", action="store_true",
                     help="split the matrices across ranks (strong scaling, one all-gather of the new "
                          "weights per step) instead of running one replica per rank")
+    ap.add_argument("--graph", action="store_true",
+                    help="time replays of one captured step (CUDA graph) instead of eager calls; "
+                         "per-kernel times then come from an eager pass after the timed region")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
@@ -276,14 +279,14 @@ def main():
         W = sm.params
         del M
 
-        def step(grads=G):
-            sm.step(grads, lr=LR, momentum=MU, nesterov=True, ns_steps=NS_STEPS, eps=EPS, stream=stream)
+        def step(grads=G, st=None):
+            sm.step(grads, lr=LR, momentum=MU, nesterov=True, ns_steps=NS_STEPS, eps=EPS, stream=st or stream)
     else:
         sm = None
 
-        def step(grads=G):
+        def step(grads=G, st=None):
             mb.muon_step(h, W, grads, M, lr=LR, momentum=MU, nesterov=True, ns_steps=NS_STEPS, eps=EPS,
-                         stream=stream)
+                         stream=st or stream)
 
     for _ in range(max(args.warmup, 0)):
         step()
@@ -295,8 +298,21 @@ def main():
         if world > 1:
             dist.barrier()
 
+    graph = None
+    if args.graph and args.shard:
+        raise SystemExit("--graph is for single-replica timing; it is not combined with --shard")
+    if args.graph:
+        mb.muon_sync(h)
+        cap = torch.cuda.Stream(dev)  # capture needs a non-default stream
+        cap.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            step(st=cap)
+        graph.replay()  # one untimed replay (part of warm-up), on the current stream
+        torch.cuda.synchronize()
+
     # ---------------- device-timed region
-    mb.muon_profile_enable(h, True)
+    mb.muon_profile_enable(h, graph is None)
     mb.muon_profile_read(h)
     gpu_uuid = None
     try:
@@ -313,13 +329,23 @@ def main():
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        step()
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
     mb.muon_sync(h)
     ms = e0.elapsed_time(e1)
+    if graph is not None:
+        # per-kernel times from eager steps (library events cannot sit inside the graph)
+        mb.muon_profile_enable(h, True)
+        mb.muon_profile_read(h)
+        for _ in range(args.steps):
+            step()
+        torch.cuda.synchronize()
     prof = mb.muon_profile_read(h)
     mb.muon_profile_enable(h, False)
     ms_max = max_over_ranks(ms, world, dev)
@@ -451,8 +477,10 @@ def main():
             "matrices_per_s": len(shapes) * args.steps * (1 if args.shard else world) / (ms_max / 1e3),
             "kernels": kernels, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+            "timing": "CUDA graph replays of one captured step" if graph is not None else "eager calls",
         }
         print(json.dumps(line), flush=True)
+    graph = None
     mb.muon_destroy(h)
     if world > 1:
         dist.barrier()
