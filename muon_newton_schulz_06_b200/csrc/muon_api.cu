@@ -220,6 +220,16 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
   P = Plan();
   P.mode = mode;
   const size_t esz = (mode == MUON_MODE_BF16) ? 2 : 4;
+  // every per-call count below must fit the 32-bit fields of the kernels' tables
+  {
+    int64_t units = 0, rows_total = 0;
+    for (int i = 0; i < n; ++i) {
+      units += ((rows[i] + kEwTile - 1) / kEwTile) * ((cols[i] + kEwTile - 1) / kEwTile);
+      rows_total += std::min(rows[i], cols[i]);
+    }
+    if (units * kWarpsPerUnit >= (int64_t(1) << 31) || rows_total >= (int64_t(1) << 31))
+      return fail(h, MUON_ERR_INVALID_ARG, "the matrices of one call are too large for one workspace");
+  }
   P.sig.resize(2 * (size_t)n);
   P.mats.resize(n);
   for (int i = 0; i < n; ++i) {

@@ -335,3 +335,23 @@ def test_cuda_graph_capture_replays_bit_exact(mb, handle):
         assert torch.equal(a, b)
     for a, b in zip(M_e, M_g):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("mode,dtype,tol", [("fp32", torch.float32, F32_TOL), ("bf16", torch.bfloat16, BF16_TOL)])
+def test_random_shapes_grouped(mb, handle, mode, dtype, tol):
+    """30 seeded random shapes (1..700 x 1..700, many sharing a group) in one call."""
+    rng = np.random.default_rng(2024)
+    shapes = [(int(rng.integers(1, 701)), int(rng.integers(1, 701))) for _ in range(24)]
+    shapes += [shapes[0], shapes[1], (shapes[2][1], shapes[2][0]), (256, 256), (512, 128), (128, 512)]
+    xs = []
+    for i, (r, c) in enumerate(shapes):
+        g = torch.Generator().manual_seed(900 + i)
+        k = min(r, c)
+        u, _ = torch.linalg.qr(torch.randn(r, k, generator=g, dtype=torch.float64))
+        v, _ = torch.linalg.qr(torch.randn(c, k, generator=g, dtype=torch.float64))
+        sv = 0.05 + 0.95 * torch.rand(k, generator=g, dtype=torch.float64)
+        xs.append(((u * sv) @ v.T).to(dtype).cuda().contiguous())
+    outs = ns_gpu(mb, handle, xs, mode)
+    for x, o in zip(xs, outs):
+        err = rel(to64(o), ns_oracle(x, [oracle.QUINTIC] * 5))
+        assert err < tol, (tuple(x.shape), err)
