@@ -13,7 +13,8 @@ value      algorithmic Newton-Schulz TFLOP (one triangle of the symmetric produc
            per step x steps, summed over ranks, / the slowest rank's device time of
            the whole steps (CUDA events on the launch stream).
 e2e        the same metric when every step also copies the gradients in from pinned
-           host memory and the updated weights back out.
+           host memory and the updated weights back out; the step is issued as four
+           calls over layer runs so the copies overlap compute (--e2e-chunks).
 roofline   the kernel with the largest share of device time, from per-launch CUDA
            events the library records on its stream during the timed steps.
 cpu_baseline  the float64 CPU oracle on a bounded sample of the same workload.
@@ -35,6 +36,7 @@ if ROOT not in sys.path:
 METRIC = "Muon step ms & NS TFLOP/s (fraction of bf16 tensor peak) per model matrix set, 1 B200"
 UNIT = "TFLOP/s"
 LR, MU, EPS, NS_STEPS = 0.02, 0.95, 1e-7, 5
+E2E_CHUNKS = 4  # calls per step in the end-to-end pipeline (transfers overlap within a step)
 WORKLOAD_TEXT = {
     1: "d8: depth-8 GPT, d_model 512, MLP 2048, 48 bf16 matrices",
     2: "d12: depth-12 GPT, d_model 768, MLP 3072, 72 bf16 matrices",
@@ -60,6 +62,9 @@ def parse():
                     help="time replays of one captured step (CUDA graph) instead of eager calls; "
                          "per-kernel times then come from an eager pass after the timed region")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=E2E_CHUNKS,
+                    help="calls per step in the end-to-end pipeline; with 1 (one call for the whole set) "
+                         "the weights' download must end before the next step starts")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     return ap.parse_args()
@@ -353,29 +358,58 @@ def main():
     value = replica_throughput(fl["algorithmic"], args.steps, 1 if args.shard else world, ms_max)
 
     # ---------------- end to end: pinned host gradients in, updated weights out, every step
-    # Step k's gradients are uploaded on a copy stream while step k-1 computes (two device
-    # gradient buffers); step k's result is staged with a device copy and downloaded on a
-    # second copy stream while step k+1 computes.  Every step still moves its full
-    # gradients in and its full weights out inside the timed region.
+    # The step is issued as E2E_CHUNKS calls over contiguous runs of matrices of about
+    # equal work (one library handle each, as a training loop would bucket its layers),
+    # so transfers overlap compute within a step as well as across steps: chunk c's
+    # gradients are uploaded on a copy stream while earlier chunks compute (two device
+    # gradient buffers alternate between steps), and chunk c's updated weights are
+    # downloaded on a second copy stream while later chunks compute.  Chunk c of the next
+    # step starts only after that download has read the weights.  Every step still moves
+    # its full gradients in and its full weights out inside the timed region.
     e2e = None
     if not args.no_e2e:
+        n_chunks = 1 if args.shard else max(1, min(args.e2e_chunks, len(W)))
+        bounds = cost.contiguous_chunks(shapes, n_chunks, NS_STEPS)
+        hc = [h] if n_chunks == 1 else [mb.muon_init(local) for _ in bounds]
         g_host = [g.cpu().pin_memory() for g in G]
         w_host = [torch.empty(w.shape, dtype=w.dtype, pin_memory=True) for w in W]
         g_dev = [G, [torch.empty_like(g) for g in G]]
-        w_stage = [torch.empty_like(w) for w in W]
         h2d_bytes = sum(x.numel() * x.element_size() for x in g_host)
         d2h_bytes = sum(x.numel() * x.element_size() for x in w_host)
         up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         ev = lambda: torch.cuda.Event()  # noqa: E731
-        g_ready, g_free = [ev(), ev()], [ev(), ev()]
-        staged, fetched = ev(), ev()
+        g_ready = [[ev() for _ in bounds] for _ in range(2)]
+        g_free = [[ev() for _ in bounds] for _ in range(2)]
+        done = [ev() for _ in bounds]
+        fetched = [ev() for _ in bounds]
 
-        def upload(k):
-            b = k % 2
+        def chunk_step(c, grads, st):
+            a, b = bounds[c]
+            if args.shard:
+                step(grads, st=st)
+            else:
+                mb.muon_step(hc[c], W[a:b], grads[a:b], M[a:b], lr=LR, momentum=MU, nesterov=True,
+                             ns_steps=NS_STEPS, eps=EPS, stream=st)
+
+        def upload(k, c):
+            a, b = bounds[c]
             with torch.cuda.stream(up):
-                for gd, gh in zip(g_dev[b], g_host):
+                for gd, gh in zip(g_dev[k % 2][a:b], g_host[a:b]):
                     gd.copy_(gh, non_blocking=True)
-                g_ready[b].record(up)
+                g_ready[k % 2][c].record(up)
+
+        def download(c):
+            a, b = bounds[c]
+            with torch.cuda.stream(down):
+                down.wait_event(done[c])
+                for wh, wd in zip(w_host[a:b], W[a:b]):
+                    wh.copy_(wd, non_blocking=True)
+                fetched[c].record(down)
+
+        # untimed pass of the chunked step (plans and workspaces of the chunk handles)
+        for c in range(n_chunks):
+            chunk_step(c, G, stream)
+        torch.cuda.synchronize()
 
         e2 = torch.cuda.Event(enable_timing=True)
         e3 = torch.cuda.Event(enable_timing=True)
@@ -384,34 +418,36 @@ def main():
         e2.record(stream)
         up.wait_event(e2)
         down.wait_event(e2)
-        fetched.record(down)
-        upload(0)
+        for c in range(n_chunks):
+            fetched[c].record(down)
+            upload(0, c)
         for k in range(args.steps):
             b = k % 2
-            if k + 1 < args.steps:
-                up.wait_event(g_free[(k + 1) % 2]) if k >= 1 else None
-                upload(k + 1)
-            stream.wait_event(g_ready[b])
-            step(g_dev[b])
-            g_free[b].record(stream)
-            stream.wait_event(fetched)            # the previous download has read the staging copy
-            for ws_, wd in zip(w_stage, W):
-                ws_.copy_(wd, non_blocking=True)
-            staged.record(stream)
-            with torch.cuda.stream(down):
-                down.wait_event(staged)
-                for wh, ws_ in zip(w_host, w_stage):
-                    wh.copy_(ws_, non_blocking=True)
-                fetched.record(down)
-        stream.wait_event(fetched)
+            for c in range(n_chunks):
+                if k + 1 < args.steps:
+                    if k >= 1:
+                        up.wait_event(g_free[(k + 1) % 2][c])
+                    upload(k + 1, c)
+                stream.wait_event(g_ready[b][c])
+                stream.wait_event(fetched[c])  # the previous step's weights of this chunk are out
+                chunk_step(c, g_dev[b], stream)
+                g_free[b][c].record(stream)
+                done[c].record(stream)
+                download(c)
+        for c in range(n_chunks):
+            stream.wait_event(fetched[c])
         e3.record(stream)
         torch.cuda.synchronize()
         ms_e2e = max_over_ranks(e2.elapsed_time(e3), world, dev)
         e2e = {"value": replica_throughput(fl["algorithmic"], args.steps, 1 if args.shard else world, ms_e2e),
                "unit": UNIT, "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
-               "ms_per_step": ms_e2e / args.steps,
-               "overlap": "upload of step k+1 and download of step k-1 run on copy streams during step k"}
-        del g_host, w_host, g_dev, w_stage
+               "ms_per_step": ms_e2e / args.steps, "chunks": n_chunks,
+               "overlap": "per chunk of matrices: upload ahead on one copy stream, download right after "
+                          "on another, both overlapping the other chunks' compute and the next step"}
+        for x in hc:
+            if x is not h:
+                mb.muon_destroy(x)
+        del g_host, w_host, g_dev
 
     # ---------------- per-kernel roofline
     pk = peaks()

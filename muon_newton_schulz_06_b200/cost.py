@@ -34,3 +34,29 @@ def elementwise_bytes(shapes: Iterable[Tuple[int, int]], param="bf16", grad="bf1
     numel = sum(r * c for r, c in shapes)
     pb, gb, wb = _BYTES[param], _BYTES[grad], _BYTES[work]
     return {"momentum_norm": numel * (gb + 4 + 4 + wb), "apply": numel * (wb + 2 * pb), "numel": numel}
+
+
+def contiguous_chunks(shapes, n_chunks: int, ns_steps: int = 5):
+    """Cut the matrix list into at most n_chunks contiguous, non-empty runs of about
+    equal algorithmic Newton-Schulz work; returns [(begin, end), ...] covering all of it.
+    Cut c goes at the matrix boundary whose running sum is closest to c/n_chunks of the
+    total (keeping every run non-empty)."""
+    shapes = list(shapes)
+    n = len(shapes)
+    if n == 0:
+        return []
+    n_chunks = max(1, min(int(n_chunks), n))
+    work = [ns_flops([sh], ns_steps)["algorithmic"] for sh in shapes]
+    prefix = [0]
+    for w in work:
+        prefix.append(prefix[-1] + w)
+    total = float(prefix[-1])
+    cuts = [0]
+    for c in range(1, n_chunks):
+        target = total * c / n_chunks
+        lo = cuts[-1] + 1                      # at least one matrix in the run before
+        hi = n - (n_chunks - c)                # at least one matrix for each later run
+        best = min(range(lo, hi + 1), key=lambda i: (abs(prefix[i] - target), i))
+        cuts.append(best)
+    cuts.append(n)
+    return [(cuts[i], cuts[i + 1]) for i in range(n_chunks)]

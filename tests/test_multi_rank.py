@@ -87,6 +87,22 @@ def test_lpt_partition_balances_the_llama_set():
     assert sharded.partition_lpt(shapes, 3) == sharded.partition_lpt(shapes, 3)  # deterministic
 
 
+def test_end_to_end_chunks_cover_the_set_in_balanced_contiguous_runs():
+    from muon_newton_schulz_06_b200.cost import contiguous_chunks, ns_flops
+    for cfg in (1, 2, 3, 4):
+        shapes = [(s.rows, s.cols) for s in synth.config_shapes(cfg)]
+        for n in (1, 2, 4, 7):
+            b = contiguous_chunks(shapes, n)
+            assert len(b) == n and b[0][0] == 0 and b[-1][1] == len(shapes)
+            assert all(x[1] == y[0] for x, y in zip(b, b[1:])) and all(e > a for a, e in b)
+            work = [ns_flops(shapes[a:e])["algorithmic"] for a, e in b]
+            assert max(work) / (sum(work) / n) < 1.25, (cfg, n, work)
+    # fewer matrices than chunks, one dominant matrix, empty list
+    assert contiguous_chunks([(4, 4)] * 3, 4) == [(0, 1), (1, 2), (2, 3)]
+    assert contiguous_chunks([(100, 100), (4, 4), (4, 4), (4, 4)], 4) == [(0, 1), (1, 2), (2, 3), (3, 4)]
+    assert contiguous_chunks([], 4) == []
+
+
 def _fake_step(params, grads, moms, lr=0.1, **kw):
     # stands in for the CUDA step on CPU: any deterministic in-place update will do
     for w, g, m in zip(params, grads, moms):
