@@ -54,9 +54,10 @@ def oracle_o(g, m):
     return o
 
 
-def test_d12_full_set(mb):
-    """Depth-12 GPT set, all 72 matrices in one call."""
-    data = synth.make_matrix_set(2, device="cuda")
+@pytest.mark.parametrize("config", [1, 2])
+def test_gpt_full_set(mb, config):
+    """Depth-8 (48 matrices) and depth-12 (72 matrices) GPT sets, each in one call."""
+    data = synth.make_matrix_set(config, device="cuda")
     W, M, scales = step_readback(mb, data)
     for i, spec in enumerate(data["specs"]):
         m_ref, _ = oracle.nesterov_momentum_f32(data["G"][i].float().cpu().numpy(), data["M"][i].cpu().numpy(),
