@@ -12,16 +12,83 @@
 //
 // One work unit is a 64 x 64 tile of the caller matrix; 256 threads each own 2 rows x 8
 // consecutive columns, so rows move as 16-byte vectors (streaming cache hints: every
-// byte is touched once per pass), and every load of a unit is issued before its stores.  Tall matrices go through a shared-memory tile to write /
-// read the transposed workspace coalesced.  The norm is deterministic: each warp of a
-// unit writes one partial sum (fixed shuffle tree), and a second small kernel adds a
-// matrix's partials in a fixed order.
+// byte is touched once per pass), and every load of a unit is issued before its stores.
+// Tall matrices go through a shared-memory tile to write / read the transposed
+// workspace coalesced.  The norm is deterministic: each warp of a unit writes one
+// partial sum (fixed shuffle tree), and a second small kernel adds a matrix's partials
+// in a fixed order.
+//
+// Matrices whose workspace copy has the caller's layout (wide, bf16 gradient, rows of
+// a multiple of 8 elements) take the bulk-copy momentum kernel instead: units of 4096
+// contiguous elements move global -> shared -> global with cp.async.bulk through a
+// 3-stage ring per CTA, so the bytes in flight are bounded by shared memory rather than
+// by registers, and the pass keeps HBM busy at the reduced SM clock of a power-capped
+// step (the tile kernel is bound by load latency there).
+#include <algorithm>
+
 #include "muon_internal.h"
 
 namespace muon {
 namespace {
 
 constexpr int kThreads = 256;
+
+// ---- bulk-copy helpers (momentum_flat_kernel)
+__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void bar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void bar_arrive_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ bool bar_try_wait(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+constexpr unsigned long long kFlatWaitNs = 2000000000ull;  // 2 s per wait
+// Bounded wait: false after kFlatWaitNs (the caller records a time-out and stops).
+__device__ __noinline__ bool bar_wait(uint64_t* b, uint32_t parity) {
+  if (bar_try_wait(b, parity)) return true;
+  const uint64_t t0 = gtimer();
+  while (!bar_try_wait(b, parity))
+    if (gtimer() - t0 > kFlatWaitNs) return false;
+  return true;
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   su32(dst)),
+               "l"(src), "r"(bytes), "r"(su32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(su32(src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+constexpr int kFlatStages = 3;
+constexpr int kFlatCompute = 128;                 // compute threads (warps 1..4)
+constexpr int kFlatThreads = 32 + kFlatCompute;   // warp 0: copy producer
+constexpr uint32_t kFlatGBytes = kFlatUnit * 2;   // bf16 gradients, then U, per stage
+constexpr uint32_t kFlatMBytes = kFlatUnit * 4;   // fp32 momentum per stage
+constexpr size_t kFlatSmem = kFlatStages * (kFlatGBytes + kFlatMBytes) + 2 * kFlatStages * sizeof(uint64_t);
 
 __device__ __forceinline__ float ld_elem(const void* p, size_t i, bool bf16) {
   return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i])
@@ -209,6 +276,123 @@ momentum_norm_kernel(const __grid_constant__ EwParams p) {
     for (int o = 16; o > 0; o >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
     if (lane == 0) p.partials[(size_t)(m.part_base + u) * kWarpsPerUnit + warp] = ssq;
   }
+}
+
+// Bulk-copy momentum pass (matrices listed in p, all with the caller's layout in the
+// workspace).  Unit u of matrix m covers elements [u*4096, min((u+1)*4096, rows*cols)).
+// Warp 0, lane 0 copies a unit's gradients and momentum into a ring stage; the 128
+// compute threads each take 8-element chunks ct, ct+128, ... of it, update M and write
+// U in place (U over the gradients), then one thread stores both back with bulk copies
+// and frees the stage once the copy engine has read it.  Each compute warp writes one
+// norm partial per unit (slots 0..3; slots 4..7 are written as zero).
+__global__ void __launch_bounds__(kFlatThreads)
+momentum_flat_kernel(const __grid_constant__ EwParams p) {
+  extern __shared__ __align__(128) uint8_t fsm[];
+  uint8_t* sg = fsm;                                 // [kFlatStages][kFlatGBytes]
+  uint8_t* smo = fsm + kFlatStages * kFlatGBytes;     // [kFlatStages][kFlatMBytes]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smo + kFlatStages * kFlatMBytes);
+  uint64_t* empty = full + kFlatStages;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < kFlatStages; ++s) {
+      bar_init(&full[s], 1);
+      bar_init(&empty[s], 1);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < p.total_units; unit += gridDim.x) {
+        const EwMat& m = p.mats[find_mat(p, unit)];
+        const size_t off = (size_t)(unit - m.unit_begin) * kFlatUnit;
+        const size_t numel = (size_t)m.rows * m.cols;
+        const uint32_t cnt = (uint32_t)(numel - off < (size_t)kFlatUnit ? numel - off : (size_t)kFlatUnit);
+        if (!bar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
+        bar_arrive_tx(&full[s], cnt * 6u);
+        bulk_load(sg + s * kFlatGBytes, reinterpret_cast<const __nv_bfloat16*>(m.grad) + off, cnt * 2u, &full[s]);
+        bulk_load(smo + s * kFlatMBytes, m.mom + off, cnt * 4u, &full[s]);
+        if (++s == kFlatStages) { s = 0; ph ^= 1u; }
+      }
+      if (!ok) {
+        atomicExch(p.status, kDevTimeout);
+        const uint64_t t0 = gtimer();  // copies already issued land within microseconds
+        while (gtimer() - t0 < 1000000ull) {
+        }
+      }
+    }
+    return;
+  }
+
+  const int ct = tid - 32;  // 0..127
+  int s = 0, prev = -1;
+  uint32_t ph = 0;
+  bool ok = true;
+  for (int unit = blockIdx.x; unit < p.total_units; unit += gridDim.x) {
+    const EwMat& m = p.mats[find_mat(p, unit)];
+    const int u = unit - m.unit_begin;
+    const size_t off = (size_t)u * kFlatUnit;
+    const size_t numel = (size_t)m.rows * m.cols;
+    const uint32_t cnt = (uint32_t)(numel - off < (size_t)kFlatUnit ? numel - off : (size_t)kFlatUnit);
+    if (!bar_wait(&full[s], ph)) { ok = false; break; }
+    uint4* gs = reinterpret_cast<uint4*>(sg + s * kFlatGBytes);
+    float4* ms = reinterpret_cast<float4*>(smo + s * kFlatMBytes);
+    float ssq = 0.f;
+#pragma unroll
+    for (int j = 0; j < kFlatUnit / 8 / kFlatCompute; ++j) {
+      const int k = ct + j * kFlatCompute;  // chunk of 8 elements
+      if ((uint32_t)k * 8u >= cnt) break;
+      const uint4 graw = gs[k];
+      const float4 m0 = ms[2 * k], m1 = ms[2 * k + 1];
+      const __nv_bfloat162* gh = reinterpret_cast<const __nv_bfloat162*>(&graw);
+      float g[8], mo[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(gh[q]);
+        g[2 * q] = f.x;
+        g[2 * q + 1] = f.y;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float gq = p.lerp ? __fmul_rn(p.omu, g[q]) : g[q];
+        const float mn = __fadd_rn(__fmul_rn(p.mu, mo[q]), gq);
+        mo[q] = mn;
+        g[q] = p.nesterov ? __fadd_rn(gq, __fmul_rn(p.mu, mn)) : mn;  // g now holds U
+        ssq = fmaf(g[q], g[q], ssq);
+      }
+      ms[2 * k] = make_float4(mo[0], mo[1], mo[2], mo[3]);
+      ms[2 * k + 1] = make_float4(mo[4], mo[5], mo[6], mo[7]);
+      uint4 ur;
+      __nv_bfloat162* uh = reinterpret_cast<__nv_bfloat162*>(&ur);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) uh[q] = __floats2bfloat162_rn(g[2 * q], g[2 * q + 1]);
+      gs[k] = ur;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+    if (lane == 0) {
+      float* part = p.partials + (size_t)(m.part_base + u) * kWarpsPerUnit;
+      part[warp - 1] = ssq;
+      part[warp - 1 + 4] = 0.f;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // smem writes -> bulk store
+    asm volatile("bar.sync 1, %0;" ::"n"(kFlatCompute) : "memory");
+    if (ct == 0) {
+      bulk_store(m.mom + off, smo + s * kFlatMBytes, cnt * 4u);
+      bulk_store(reinterpret_cast<__nv_bfloat16*>(m.work) + off, sg + s * kFlatGBytes, cnt * 2u);
+      bulk_commit();
+      bulk_wait_read1();  // the previous unit's stores have read their stage
+      if (prev >= 0) bar_arrive(&empty[prev]);
+    }
+    prev = s;
+    if (++s == kFlatStages) { s = 0; ph ^= 1u; }
+  }
+  if (ct == 0) bulk_wait_all();
+  if (!ok && ct == 0) atomicExch(p.status, kDevTimeout);
 }
 
 // scale[gid] = 1 / (sqrt(sum of the matrix's partials) + eps): one block per matrix,
@@ -434,6 +618,42 @@ cudaError_t launch_momentum_norm(const EwParams& p, bool work_f32, int grid, cud
   if (e != cudaSuccess) return e;
   norm_finalize_kernel<<<p.n_mats, kThreads, 0, st>>>(p);
   return cudaGetLastError();
+}
+
+cudaError_t launch_momentum_split(const EwParams& flat, const EwParams& rest, const EwParams& all, int sm_count,
+                                  int* launches, cudaStream_t st) {
+  *launches = 0;
+  if (flat.n_mats > 0 && flat.total_units > 0) {
+    static bool smem_set[64] = {};  // per device
+    int dev = 0;
+    cudaError_t e0 = cudaGetDevice(&dev);
+    if (e0 != cudaSuccess) return e0;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!smem_set[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(momentum_flat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)kFlatSmem);
+      if (e != cudaSuccess) return e;
+      smem_set[dev] = true;
+    }
+    const int grid = std::max(1, std::min(flat.total_units, 2 * sm_count));
+    momentum_flat_kernel<<<grid, kFlatThreads, kFlatSmem, st>>>(flat);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ++*launches;
+  }
+  if (rest.n_mats > 0 && rest.total_units > 0) {
+    const int grid = std::max(1, std::min(rest.total_units, sm_count * 8));
+    momentum_norm_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(rest);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ++*launches;
+  }
+  if (all.n_mats > 0) {
+    norm_finalize_kernel<<<all.n_mats, kThreads, 0, st>>>(all);
+    ++*launches;
+    return cudaGetLastError();
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_normuon(const EwParams& p, bool work_f32, int grid, cudaStream_t st) {

@@ -423,6 +423,46 @@ void* work_ptr(muon_handle* h, const MatPlan& m, int buf) {
   return h->ws + g.off_x[buf] + (size_t)m.idx * g.s * g.ld_x * esz;
 }
 
+// Momentum pass of one batch in bf16 mode: matrices whose workspace copy has the caller's
+// layout (not transposed, bf16 gradient, rows a multiple of 8 elements, 16-byte
+// aligned buffers) go to the bulk-copy kernel in units of kFlatUnit contiguous elements;
+// the others to the tile kernel.  The norm finalize sees every matrix with the unit
+// count of its kernel.
+cudaError_t launch_momentum_bf16(muon_handle* h, const EwParams& ep, int* launches, cudaStream_t st) {
+  EwParams* flat = new EwParams(ep);
+  EwParams* rest = new EwParams(ep);
+  EwParams* all = new EwParams(ep);
+  flat->n_mats = rest->n_mats = 0;
+  int uf = 0, ur = 0;
+  for (int j = 0; j < ep.n_mats; ++j) {
+    const EwMat& m = ep.mats[j];
+    const bool aligned = (reinterpret_cast<uintptr_t>(m.grad) % 16 == 0) &&
+                         (reinterpret_cast<uintptr_t>(m.mom) % 16 == 0) &&
+                         (reinterpret_cast<uintptr_t>(m.work) % 16 == 0);
+    const bool is_flat = !m.transposed && m.grad_bf16 && m.cols % 8 == 0 && m.ld == m.cols && aligned;
+    EwMat e = m;
+    if (is_flat) {
+      const int64_t numel = (int64_t)m.rows * m.cols;
+      e.n_units = (int32_t)((numel + kFlatUnit - 1) / kFlatUnit);
+      e.unit_begin = uf;
+      uf += e.n_units;
+      flat->mats[flat->n_mats++] = e;
+    } else {
+      e.unit_begin = ur;
+      ur += e.n_units;
+      rest->mats[rest->n_mats++] = e;
+    }
+    all->mats[j].n_units = e.n_units;
+  }
+  flat->total_units = uf;
+  rest->total_units = ur;
+  cudaError_t err = launch_momentum_split(*flat, *rest, *all, h->sm_count, launches, st);
+  delete flat;
+  delete rest;
+  delete all;
+  return err;
+}
+
 muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, int pass, int out_kind,
                                int work_buf, const CallOpts& o, cudaStream_t st) {
   const bool momentum_pass = pass == kPassMomentum;
@@ -449,6 +489,7 @@ muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, i
     ep->eps = eps;
     ep->partials = reinterpret_cast<float*>(h->ws + P.off_partials);
     ep->scale = reinterpret_cast<float*>(h->ws + P.off_scale);
+    ep->status = h->dev_status;
     int units = 0;
     for (int j = 0; j < ep->n_mats; ++j) {
       const int i = b + j;
@@ -480,16 +521,22 @@ muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, i
     }
     ep->total_units = units;
     const int grid = std::max(1, std::min(units, h->sm_count * 8));
+    int launches = pass == kPassOut ? 1 : 2;
     prof_begin(h, st);
-    cudaError_t err = pass == kPassMomentum ? launch_momentum_norm(*ep, f32, grid, st)
-                      : pass == kPassNormuon ? launch_normuon(*ep, f32, h->sm_count * 8, st)
-                                             : launch_apply(*ep, f32, out_kind, grid, st);
+    cudaError_t err;
+    if (pass == kPassMomentum && ep->use_momentum && !f32) {
+      err = launch_momentum_bf16(h, *ep, &launches, st);
+    } else {
+      err = pass == kPassMomentum ? launch_momentum_norm(*ep, f32, grid, st)
+            : pass == kPassNormuon ? launch_normuon(*ep, f32, h->sm_count * 8, st)
+                                   : launch_apply(*ep, f32, out_kind, grid, st);
+    }
     prof_end(h, pass == kPassMomentum ? MUON_KIND_MOMENTUM_NORM : MUON_KIND_APPLY, st);
     delete ep;
     if (err != cudaSuccess)
       return cuda_fail(h, err, pass == kPassMomentum ? "momentum/norm launch"
                                : pass == kPassNormuon ? "NorMuon launch" : "apply launch");
-    h->last_launches += pass == kPassOut ? 1 : 2;
+    h->last_launches += launches;
   }
   return MUON_OK;
 }

@@ -23,6 +23,11 @@ constexpr int kMaxMatsPerLaunch = 192;
 // Square tile of one elementwise work unit, and the norm partials it writes (one per warp).
 constexpr int kEwTile = 64;
 constexpr int kWarpsPerUnit = 8;
+// Unit of the bulk-copy momentum pass: a contiguous run of elements of a matrix whose
+// workspace copy has the caller's layout (wide, row length a multiple of 8).  It holds
+// as many elements as a 64 x 64 tile, so a matrix never has more of these units than
+// tiles and the partials array sized for tiles holds them.
+constexpr int kFlatUnit = kEwTile * kEwTile;
 
 struct EwMat {
   void* param;          // caller matrix: param (apply), or x_in (normalise-only)
@@ -63,6 +68,7 @@ struct EwParams {
   float eps;
   float* partials;      // per (unit, warp) sum of squares
   float* scale;         // per-matrix 1/(||U||_F + eps)
+  int* status;          // device status word (bounded waits record a time-out here)
 };
 
 enum EwOut : int { kEwApply = 0, kEwExport = 1 };
@@ -74,6 +80,12 @@ cudaError_t launch_normuon(const EwParams& p, bool work_f32, int grid, cudaStrea
 // Launchers (k_elementwise.cu).  work_f32 selects the workspace element type.
 // launch_momentum_norm enqueues two kernels: the pass and the per-matrix norm finalize.
 cudaError_t launch_momentum_norm(const EwParams& p, bool work_f32, int grid, cudaStream_t st);
+// Momentum pass split by matrix kind (bf16 workspace): `flat` lists the matrices run by
+// the bulk-copy kernel (units of kFlatUnit contiguous elements), `rest` those run by the
+// tile kernel; `all` lists every matrix with its unit count for the norm finalize.
+// Empty lists are skipped.  Returns the number of kernels enqueued in *launches.
+cudaError_t launch_momentum_split(const EwParams& flat, const EwParams& rest, const EwParams& all, int sm_count,
+                                  int* launches, cudaStream_t st);
 cudaError_t launch_apply(const EwParams& p, bool work_f32, int out_kind, int grid, cudaStream_t st);
 
 // ----------------------------------------------------------------- tensor-core engine
