@@ -18,12 +18,14 @@
 // partial sum (fixed shuffle tree), and a second small kernel adds a matrix's partials
 // in a fixed order.
 //
-// Matrices whose workspace copy has the caller's layout (wide, bf16 gradient, rows of
-// a multiple of 8 elements) take the bulk-copy momentum kernel instead: units of 4096
-// contiguous elements move global -> shared -> global with cp.async.bulk through a
-// 3-stage ring per CTA, so the bytes in flight are bounded by shared memory rather than
-// by registers, and the pass keeps HBM busy at the reduced SM clock of a power-capped
-// step (the tile kernel is bound by load latency there).
+// In bf16 mode the momentum pass moves data with the copy engine instead: wide matrices
+// (workspace copy in the caller's layout) in units of 4096 contiguous elements through
+// cp.async.bulk, tall ones in 64 x 64 tiles through tensor maps (cp.async.bulk.tensor,
+// 128-byte swizzle, transposed in shared memory), each through a 3-stage ring per CTA.
+// The bytes in flight are then bounded by shared memory rather than by registers, and
+// the pass keeps HBM busy at the reduced SM clock of a power-capped step (the register
+// tile kernel is bound by load latency there).  Matrices that fit neither (fp32
+// gradients, unaligned rows) keep the register tile kernel.
 #include <algorithm>
 
 #include "muon_internal.h"
@@ -79,6 +81,18 @@ __device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t 
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(su32(src)), "r"(bytes)
                : "memory");
 }
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(su32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(su32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(x),
+               "r"(y), "r"(su32(src))
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -89,6 +103,14 @@ constexpr int kFlatThreads = 32 + kFlatCompute;   // warp 0: copy producer
 constexpr uint32_t kFlatGBytes = kFlatUnit * 2;   // bf16 gradients, then U, per stage
 constexpr uint32_t kFlatMBytes = kFlatUnit * 4;   // fp32 momentum per stage
 constexpr size_t kFlatSmem = kFlatStages * (kFlatGBytes + kFlatMBytes) + 2 * kFlatStages * sizeof(uint64_t);
+// TMA tile pass: per stage a gradient tile (8 KB), a momentum tile (two 32-column halves,
+// 16 KB) and the transposed U tile (8 KB), each 1024-byte aligned for the swizzle.
+constexpr uint32_t kTileStageBytes = kFlatGBytes + kFlatMBytes + kFlatGBytes;
+constexpr size_t kTileSmem = 1024 + kFlatStages * kTileStageBytes + 2 * kFlatStages * sizeof(uint64_t);
+
+// Byte offset of the 16-byte chunk q of row r in a tile with 128-byte rows and the
+// 128-byte swizzle (chunk index XOR row mod 8), as the tensor maps lay it out.
+__device__ __forceinline__ uint32_t swz128(int r, int q) { return (uint32_t)(r * 128 + ((q ^ (r & 7)) << 4)); }
 
 __device__ __forceinline__ float ld_elem(const void* p, size_t i, bool bf16) {
   return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i])
@@ -152,7 +174,8 @@ __device__ __forceinline__ void st8_dyn(void* p, size_t i, const float* v, bool 
 }
 
 // Matrix of a launch-wide work unit (binary search over unit_begin).
-__device__ __forceinline__ int find_mat(const EwParams& p, int unit) {
+template <typename P>
+__device__ __forceinline__ int find_mat(const P& p, int unit) {
   int lo = 0, hi = p.n_mats - 1;
   while (lo < hi) {
     int mid = (lo + hi + 1) >> 1;
@@ -395,6 +418,130 @@ momentum_flat_kernel(const __grid_constant__ EwParams p) {
   if (!ok && ct == 0) atomicExch(p.status, kDevTimeout);
 }
 
+// TMA momentum pass of tall matrices (p lists them; unit u of matrix m is the 64 x 64 tile
+// (u / tiles_c, u % tiles_c) of the caller matrix).  Warp 0, lane 0 loads the gradient
+// and momentum tiles through the matrix's tensor maps (out-of-range parts read as
+// zero); compute thread ct owns row ct mod 64 of the tile, columns 32*(ct/64) ..+31:
+// it updates M in place and writes U transposed into the U tile (U^T row c, column r),
+// then one thread stores M and U^T through the maps (clipped at the matrix edge).
+// 128-byte swizzled tiles keep both the row reads and the transposed writes free of
+// bank conflicts.  Norm partials as in momentum_flat_kernel.
+__global__ void __launch_bounds__(kFlatThreads)
+momentum_tile_tma_kernel(const __grid_constant__ EwTiledParams p) {
+  extern __shared__ uint8_t tsm_raw[];
+  uint8_t* tsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(tsm + kFlatStages * kTileStageBytes);
+  uint64_t* empty = full + kFlatStages;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < kFlatStages; ++s) {
+      bar_init(&full[s], 1);
+      bar_init(&empty[s], 1);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  auto g_tile = [&](int s) { return tsm + s * kTileStageBytes; };
+  auto m_tile = [&](int s) { return tsm + s * kTileStageBytes + kFlatGBytes; };  // [2][64 rows][128 B]
+  auto u_tile = [&](int s) { return tsm + s * kTileStageBytes + kFlatGBytes + kFlatMBytes; };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < p.total_units; unit += gridDim.x) {
+        const EwMat& m = p.mats[find_mat(p, unit)];
+        const int u = unit - m.unit_begin;
+        const int r0 = (u / m.tiles_c) * kEwTile, c0 = (u % m.tiles_c) * kEwTile;
+        const CUtensorMap* maps = &p.maps[kEwMapsPerMat * find_mat(p, unit)];
+        if (!bar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
+        bar_arrive_tx(&full[s], kFlatGBytes + kFlatMBytes);
+        tma_load_2d(g_tile(s), &maps[0], c0, r0, &full[s]);
+        tma_load_2d(m_tile(s), &maps[1], c0, r0, &full[s]);
+        tma_load_2d(m_tile(s) + kFlatMBytes / 2, &maps[1], c0 + 32, r0, &full[s]);
+        if (++s == kFlatStages) { s = 0; ph ^= 1u; }
+      }
+      if (!ok) {
+        atomicExch(p.status, kDevTimeout);
+        const uint64_t t0 = gtimer();  // copies already issued land within microseconds
+        while (gtimer() - t0 < 1000000ull) {
+        }
+      }
+    }
+    return;
+  }
+
+  const int ct = tid - 32;   // 0..127
+  const int r = ct & 63;     // tile row of this thread
+  const int h = ct >> 6;     // column half: columns 32h .. 32h+31
+  int s = 0, prev = -1;
+  uint32_t ph = 0;
+  bool ok = true;
+  for (int unit = blockIdx.x; unit < p.total_units; unit += gridDim.x) {
+    const EwMat& m = p.mats[find_mat(p, unit)];
+    const int u = unit - m.unit_begin;
+    const int r0 = (u / m.tiles_c) * kEwTile, c0 = (u % m.tiles_c) * kEwTile;
+    if (!bar_wait(&full[s], ph)) { ok = false; break; }
+    uint8_t* gt = g_tile(s);
+    uint8_t* mt = m_tile(s) + h * (kFlatMBytes / 2);
+    uint8_t* ut = u_tile(s);
+    float ssq = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // 8 columns 32h + 8i .. +7
+      const uint4 graw = *reinterpret_cast<const uint4*>(gt + swz128(r, 4 * h + i));
+      float4* mp0 = reinterpret_cast<float4*>(mt + swz128(r, 2 * i));
+      float4* mp1 = reinterpret_cast<float4*>(mt + swz128(r, 2 * i + 1));
+      const float4 m0 = *mp0, m1 = *mp1;
+      const __nv_bfloat162* gh = reinterpret_cast<const __nv_bfloat162*>(&graw);
+      float g[8], mo[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(gh[q]);
+        g[2 * q] = f.x;
+        g[2 * q + 1] = f.y;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float gq = p.lerp ? __fmul_rn(p.omu, g[q]) : g[q];
+        const float mn = __fadd_rn(__fmul_rn(p.mu, mo[q]), gq);
+        mo[q] = mn;
+        g[q] = p.nesterov ? __fadd_rn(gq, __fmul_rn(p.mu, mn)) : mn;  // g now holds U
+        ssq = fmaf(g[q], g[q], ssq);
+      }
+      *mp0 = make_float4(mo[0], mo[1], mo[2], mo[3]);
+      *mp1 = make_float4(mo[4], mo[5], mo[6], mo[7]);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {  // U^T row c = 32h + 8i + q, column r
+        const int c = 32 * h + 8 * i + q;
+        *reinterpret_cast<__nv_bfloat16*>(ut + swz128(c, r >> 3) + ((r & 7) << 1)) = __float2bfloat16_rn(g[q]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+    if (lane == 0) {
+      float* part = p.partials + (size_t)(m.part_base + u) * kWarpsPerUnit;
+      part[warp - 1] = ssq;
+      part[warp - 1 + 4] = 0.f;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // smem writes -> tensor store
+    asm volatile("bar.sync 1, %0;" ::"n"(kFlatCompute) : "memory");
+    if (ct == 0) {
+      const CUtensorMap* maps = &p.maps[kEwMapsPerMat * find_mat(p, unit)];
+      tma_store_2d(&maps[1], m_tile(s), c0, r0);
+      tma_store_2d(&maps[1], m_tile(s) + kFlatMBytes / 2, c0 + 32, r0);
+      tma_store_2d(&maps[2], ut, r0, c0);
+      bulk_commit();
+      bulk_wait_read1();  // the previous unit's stores have read their stage
+      if (prev >= 0) bar_arrive(&empty[prev]);
+    }
+    prev = s;
+    if (++s == kFlatStages) { s = 0; ph ^= 1u; }
+  }
+  if (ct == 0) bulk_wait_all();
+  if (!ok && ct == 0) atomicExch(p.status, kDevTimeout);
+}
+
 // scale[gid] = 1 / (sqrt(sum of the matrix's partials) + eps): one block per matrix,
 // fixed summation order (strided per thread, then a fixed tree), in double.
 __global__ void __launch_bounds__(kThreads)
@@ -620,21 +767,32 @@ cudaError_t launch_momentum_norm(const EwParams& p, bool work_f32, int grid, cud
   return cudaGetLastError();
 }
 
-cudaError_t launch_momentum_split(const EwParams& flat, const EwParams& rest, const EwParams& all, int sm_count,
-                                  int* launches, cudaStream_t st) {
+cudaError_t launch_momentum_split(const EwParams& flat, const EwTiledParams* tiled, int n_tiled, const EwParams& rest,
+                                  const EwParams& all, int sm_count, int* launches, cudaStream_t st) {
   *launches = 0;
+  static bool smem_set[64] = {};  // per device
+  int dev = 0;
+  cudaError_t e0 = cudaGetDevice(&dev);
+  if (e0 != cudaSuccess) return e0;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!smem_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(momentum_flat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kFlatSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(momentum_tile_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kTileSmem);
+    if (e != cudaSuccess) return e;
+    smem_set[dev] = true;
+  }
+  for (int t = 0; t < n_tiled; ++t) {
+    if (tiled[t].n_mats == 0 || tiled[t].total_units == 0) continue;
+    const int grid = std::max(1, std::min(tiled[t].total_units, 2 * sm_count));
+    momentum_tile_tma_kernel<<<grid, kFlatThreads, kTileSmem, st>>>(tiled[t]);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ++*launches;
+  }
   if (flat.n_mats > 0 && flat.total_units > 0) {
-    static bool smem_set[64] = {};  // per device
-    int dev = 0;
-    cudaError_t e0 = cudaGetDevice(&dev);
-    if (e0 != cudaSuccess) return e0;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!smem_set[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(momentum_flat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)kFlatSmem);
-      if (e != cudaSuccess) return e;
-      smem_set[dev] = true;
-    }
     const int grid = std::max(1, std::min(flat.total_units, 2 * sm_count));
     momentum_flat_kernel<<<grid, kFlatThreads, kFlatSmem, st>>>(flat);
     cudaError_t e = cudaGetLastError();

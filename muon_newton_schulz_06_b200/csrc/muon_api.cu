@@ -92,6 +92,10 @@ struct muon_handle {
   bool status_pending = false;
   Plan plan;
   TcApplyTable* apply_table = nullptr;  // host staging of the fused weight-update table
+  // TMA momentum pass of tall matrices: the tensor maps of each caller matrix and the
+  // pointers they were encoded for (grad, momentum, workspace); cleared with the plan
+  std::vector<CUtensorMap> ewmap;
+  std::vector<const void*> ewmap_key;
   // per-launch timing (muon_profile_enable)
   bool profiling = false;
   std::vector<cudaEvent_t> ev_free;
@@ -218,6 +222,8 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
                        cudaStream_t st) {
   Plan& P = h->plan;
   P = Plan();
+  h->ewmap.clear();  // the momentum-pass tensor maps describe the old plan's buffers
+  h->ewmap_key.clear();
   P.mode = mode;
   const size_t esz = (mode == MUON_MODE_BF16) ? 2 : 4;
   // every per-call count below must fit the 32-bit fields of the kernels' tables
@@ -423,30 +429,89 @@ void* work_ptr(muon_handle* h, const MatPlan& m, int buf) {
   return h->ws + g.off_x[buf] + (size_t)m.idx * g.s * g.ld_x * esz;
 }
 
-// Momentum pass of one batch in bf16 mode: matrices whose workspace copy has the caller's
-// layout (not transposed, bf16 gradient, rows a multiple of 8 elements, 16-byte
-// aligned buffers) go to the bulk-copy kernel in units of kFlatUnit contiguous elements;
-// the others to the tile kernel.  The norm finalize sees every matrix with the unit
-// count of its kernel.
-cudaError_t launch_momentum_bf16(muon_handle* h, const EwParams& ep, int* launches, cudaStream_t st) {
+// Tensor maps of the TMA momentum pass for caller matrix i (tall, bf16 gradient, row
+// length a multiple of 8): gradient and momentum in the caller's layout, workspace X =
+// U^T (s x L with leading dimension ld).  Written into the handle's cache at slot i.
+CUresult encode_ew_maps(muon_handle* h, int i, const EwMat& m) {
+  CUtensorMap* out = h->ewmap.data() + (size_t)i * kEwMapsPerMat;
+  const cuuint32_t estr[2] = {1, 1};
+  auto enc = [&](CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                 uint64_t stride_bytes, uint32_t box_inner) {
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {stride_bytes};
+    const cuuint32_t box[2] = {box_inner, (cuuint32_t)kEwTile};
+    return h->encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  };
+  const uint64_t rows = (uint64_t)m.rows, cols = (uint64_t)m.cols;
+  CUresult r = enc(&out[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, m.grad, cols, rows, cols * 2, 64);
+  if (r == CUDA_SUCCESS) r = enc(&out[1], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, m.mom, cols, rows, cols * 4, 32);
+  if (r == CUDA_SUCCESS) r = enc(&out[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, m.work, rows, cols, (uint64_t)m.ld * 2, 64);
+  return r;
+}
+
+// Momentum pass of one batch in bf16 mode (batch = caller matrices b .. b + n_mats - 1).
+// Wide matrices whose workspace copy has the caller's layout go to the bulk-copy kernel
+// in units of kFlatUnit contiguous elements; tall ones to the TMA tile kernel, whose
+// tensor maps travel by value with the launch (re-encoded only for matrices whose
+// pointers changed); matrices that fit neither (fp32 gradients, row lengths not a
+// multiple of 8, unaligned buffers) to the register tile kernel.  The norm finalize
+// sees every matrix with the unit count of its kernel.
+cudaError_t launch_momentum_bf16(muon_handle* h, const EwParams& ep, int b, int* launches, cudaStream_t st) {
+  const size_t n_all = h->plan.mats.size();
+  if (h->ewmap.size() != n_all * kEwMapsPerMat) {
+    h->ewmap.assign(n_all * kEwMapsPerMat, CUtensorMap{});
+    h->ewmap_key.assign(n_all * kEwMapsPerMat, nullptr);
+  }
   EwParams* flat = new EwParams(ep);
   EwParams* rest = new EwParams(ep);
   EwParams* all = new EwParams(ep);
+  const int max_tiled = (ep.n_mats + kMaxTiledPerLaunch - 1) / kMaxTiledPerLaunch;
+  EwTiledParams* tiled = new EwTiledParams[max_tiled > 0 ? max_tiled : 1]();
+  int n_tiled = 0;
   flat->n_mats = rest->n_mats = 0;
   int uf = 0, ur = 0;
+  cudaError_t err = cudaSuccess;
   for (int j = 0; j < ep.n_mats; ++j) {
     const EwMat& m = ep.mats[j];
+    const int i = b + j;  // caller index: cache slot of this matrix's maps
     const bool aligned = (reinterpret_cast<uintptr_t>(m.grad) % 16 == 0) &&
                          (reinterpret_cast<uintptr_t>(m.mom) % 16 == 0) &&
                          (reinterpret_cast<uintptr_t>(m.work) % 16 == 0);
-    const bool is_flat = !m.transposed && m.grad_bf16 && m.cols % 8 == 0 && m.ld == m.cols && aligned;
+    const bool eligible = m.grad_bf16 && m.cols % 8 == 0 && aligned;
     EwMat e = m;
-    if (is_flat) {
+    if (eligible && !m.transposed && m.ld == m.cols) {
       const int64_t numel = (int64_t)m.rows * m.cols;
       e.n_units = (int32_t)((numel + kFlatUnit - 1) / kFlatUnit);
       e.unit_begin = uf;
       uf += e.n_units;
       flat->mats[flat->n_mats++] = e;
+    } else if (eligible && m.transposed) {
+      const void** key = h->ewmap_key.data() + (size_t)i * kEwMapsPerMat;
+      if (key[0] != m.grad || key[1] != m.mom || key[2] != m.work) {
+        if (encode_ew_maps(h, i, m) != CUDA_SUCCESS) {
+          err = cudaErrorInvalidValue;
+          break;
+        }
+        key[0] = m.grad;
+        key[1] = m.mom;
+        key[2] = m.work;
+      }
+      if (n_tiled == 0 || tiled[n_tiled - 1].n_mats == kMaxTiledPerLaunch) {
+        EwTiledParams& tp = tiled[n_tiled++];
+        tp.mu = ep.mu;
+        tp.nesterov = ep.nesterov;
+        tp.lerp = ep.lerp;
+        tp.omu = ep.omu;
+        tp.partials = ep.partials;
+        tp.status = ep.status;
+      }
+      EwTiledParams& tp = tiled[n_tiled - 1];
+      std::memcpy(&tp.maps[tp.n_mats * kEwMapsPerMat], &h->ewmap[(size_t)i * kEwMapsPerMat],
+                  kEwMapsPerMat * sizeof(CUtensorMap));
+      e.unit_begin = tp.total_units;
+      tp.total_units += e.n_units;
+      tp.mats[tp.n_mats++] = e;
     } else {
       e.unit_begin = ur;
       ur += e.n_units;
@@ -456,10 +521,11 @@ cudaError_t launch_momentum_bf16(muon_handle* h, const EwParams& ep, int* launch
   }
   flat->total_units = uf;
   rest->total_units = ur;
-  cudaError_t err = launch_momentum_split(*flat, *rest, *all, h->sm_count, launches, st);
+  if (err == cudaSuccess) err = launch_momentum_split(*flat, tiled, n_tiled, *rest, *all, h->sm_count, launches, st);
   delete flat;
   delete rest;
   delete all;
+  delete[] tiled;
   return err;
 }
 
@@ -525,7 +591,7 @@ muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, i
     prof_begin(h, st);
     cudaError_t err;
     if (pass == kPassMomentum && ep->use_momentum && !f32) {
-      err = launch_momentum_bf16(h, *ep, &launches, st);
+      err = launch_momentum_bf16(h, *ep, b, &launches, st);
     } else {
       err = pass == kPassMomentum ? launch_momentum_norm(*ep, f32, grid, st)
             : pass == kPassNormuon ? launch_normuon(*ep, f32, h->sm_count * 8, st)
@@ -982,6 +1048,7 @@ muon_status muon_destroy(muon_handle_t h) {
     if (h->dev_status) cudaFree(h->dev_status);
     if (h->host_status) cudaFreeHost(h->host_status);
     if (h->status_event) cudaEventDestroy(h->status_event);
+
     for (auto& p : h->ev_pending) {
       cudaEventDestroy(p.a);
       cudaEventDestroy(p.b);

@@ -70,6 +70,26 @@ struct EwParams {
   float* scale;         // per-matrix 1/(||U||_F + eps)
   int* status;          // device status word (bounded waits record a time-out here)
 };
+static_assert(sizeof(EwParams) <= 32764, "elementwise parameters must fit the kernel parameter space");
+
+// TMA momentum pass of tall matrices (rows > cols): per matrix three tensor maps, passed
+// by value with the launch: gradient (bf16, 64 x 64 boxes), momentum (fp32, 32 x 64
+// boxes) and workspace X = U^T (bf16, 64 x 64 boxes), all with the 128-byte swizzle.
+constexpr int kEwMapsPerMat = 3;
+constexpr int kMaxTiledPerLaunch = 32;
+struct __align__(64) EwTiledParams {
+  CUtensorMap maps[kMaxTiledPerLaunch * kEwMapsPerMat];
+  EwMat mats[kMaxTiledPerLaunch];
+  int n_mats;
+  int total_units;
+  float mu;
+  int nesterov;
+  int lerp;
+  float omu;
+  float* partials;
+  int* status;
+};
+static_assert(sizeof(EwTiledParams) <= 32764, "tiled momentum parameters must fit the kernel parameter space");
 
 enum EwOut : int { kEwApply = 0, kEwExport = 1 };
 
@@ -80,12 +100,14 @@ cudaError_t launch_normuon(const EwParams& p, bool work_f32, int grid, cudaStrea
 // Launchers (k_elementwise.cu).  work_f32 selects the workspace element type.
 // launch_momentum_norm enqueues two kernels: the pass and the per-matrix norm finalize.
 cudaError_t launch_momentum_norm(const EwParams& p, bool work_f32, int grid, cudaStream_t st);
-// Momentum pass split by matrix kind (bf16 workspace): `flat` lists the matrices run by
-// the bulk-copy kernel (units of kFlatUnit contiguous elements), `rest` those run by the
+// Momentum pass split by matrix kind (bf16 workspace): `flat` lists the wide matrices run
+// by the bulk-copy kernel (units of kFlatUnit contiguous elements), `tiled[0..n_tiled)`
+// the tall ones run by the TMA tile kernel (64 x 64 tiles through tensor maps,
+// transposed in shared memory; one launch per entry), `rest` those run by the register
 // tile kernel; `all` lists every matrix with its unit count for the norm finalize.
 // Empty lists are skipped.  Returns the number of kernels enqueued in *launches.
-cudaError_t launch_momentum_split(const EwParams& flat, const EwParams& rest, const EwParams& all, int sm_count,
-                                  int* launches, cudaStream_t st);
+cudaError_t launch_momentum_split(const EwParams& flat, const EwTiledParams* tiled, int n_tiled, const EwParams& rest,
+                                  const EwParams& all, int sm_count, int* launches, cudaStream_t st);
 cudaError_t launch_apply(const EwParams& p, bool work_f32, int out_kind, int grid, cudaStream_t st);
 
 // ----------------------------------------------------------------- tensor-core engine
