@@ -191,6 +191,34 @@ def test_apply_exact_and_momentum_bitexact(mb, handle):
         assert rel(to64(O[i]), o_ref) < BF16_TOL, i
 
 
+@pytest.mark.parametrize("lerp", [False, True])
+def test_copy_engine_momentum_pass_edges(mb, handle, lerp):
+    """bf16 momentum pass through the copy engine at its edges: tall matrices with ragged
+    64 x 64 tiles (tensor-map path: zero fill on load, clipping on store, transposed
+    workspace), wide matrices whose element count leaves a partial last 4096-element
+    unit (bulk-copy path), and one matrix per path in a single grouped call.  Momentum
+    bit-exact; O within the bf16 bar."""
+    shapes = [(1000, 136), (700, 8), (130, 72), (2100, 520), (5, 1000), (100, 808), (3, 8), (40, 4104)]
+    gen = torch.Generator().manual_seed(11)
+    G32 = [torch.randn(r, c, generator=gen) for r, c in shapes]
+    M32 = [0.01 * torch.randn(r, c, generator=gen) for r, c in shapes]
+    G = [g.to(torch.bfloat16).cuda() for g in G32]
+    M = [m.cuda() for m in M32]
+    W = [torch.zeros(r, c, device="cuda") for r, c in shapes]
+    kw = {"momentum_form": "lerp"} if lerp else {}
+    mb.muon_step_ex(handle, W, G, M, lr=1.0, momentum=0.95, nesterov=True, **kw)
+    torch.cuda.synchronize()
+    mb.muon_sync(handle)
+    for i, (r, c) in enumerate(shapes):
+        g = G[i].float().cpu().numpy()
+        m_ref, _ = oracle.nesterov_momentum_f32(g, M32[i].numpy(), 0.95, True, lerp=lerp)
+        assert np.array_equal(M[i].cpu().numpy(), m_ref), (r, c)
+        _, _, o_ref = oracle.muon_step_matrix(np.zeros((r, c)), g, M32[i].numpy(), lr=1.0, mu=0.95,
+                                              nesterov=True, eps=1e-7, lerp=lerp)
+        o = -to64(W[i]) / oracle.update_scale(r, c)
+        assert rel(o, o_ref) < BF16_TOL, ((r, c), rel(o, o_ref))
+
+
 def test_grouped_step_matches_single_matrix_calls(mb, handle):
     """Packing many shapes into one grouped launch gives the same bits as one call per matrix."""
     data = synth.make_matrix_set(1, layers=[0])
