@@ -1,11 +1,13 @@
 // Host side of the Muon C ABI: argument checks, the plan (shape groups, workspace
 // layout, tile lists, TMA tensor maps) and the stream-ordered launch sequence
 //
-//   momentum_norm + norm finalize -> { Gram -> Poly -> Update } x ns_steps
+//   momentum pass + norm finalize -> { Gram -> Poly -> Update } x ns_steps
 //
 // where the last Update also applies W -= lr*scale*O in its epilogue (bf16 mode; in fp32
 // mode, and for the Newton-Schulz entry point, a separate apply / export pass follows).
-// 17 launches for five steps when the shapes fit one launch per phase.  Matrices
+// In bf16 mode the momentum pass is a bulk-copy kernel for wide matrices and a TMA tile
+// kernel for tall ones (register tile kernel otherwise): 18 launches for five steps
+// when a set has both orientations and the shapes fit one launch per phase.  Matrices
 // of equal wide-orientation shape (s, L) = (min(r,c), max(r,c)) are stacked into one
 // group, the device analogue of the per-shape-group stacking of the momentum
 // buffers that the autoresearch train.py review describes for MuonAdamW.
