@@ -381,3 +381,34 @@ def test_normuon_rows_vs_columns_by_aspect():
     a, _ = oracle.normuon_rescale(o, np.full(4, 0.3), 0.5, 1e-6)
     b, _ = oracle.normuon_rescale(o.T, np.full(4, 0.3), 0.5, 1e-6)
     assert np.allclose(a, b.T, rtol=1e-14)
+
+
+def test_normalisation_adds_eps_to_the_norm():
+    """X0 = U / (||U||_F + eps): with ||U|| = 5 and eps = 1 the divisor is 6, not
+    sqrt(25 + 1) (eps added to the squared norm) nor 5 (eps ignored)."""
+    x0 = oracle.frobenius_normalise(np.array([[3.0, 4.0]]), 1.0)
+    assert np.allclose(x0, [[0.5, 4.0 / 6.0]], rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("tall", [False, True])
+def test_step_rank_one_closed_form(tall):
+    """Whole step on a rank-one gradient, closed form.  With M = 0 and Nesterov, M' = G and
+    U = (1 + mu) G; X0 = U / (||U|| + eps) has the single singular value
+    s = (1 + mu)||G|| / ((1 + mu)||G|| + eps) and the same singular vectors, so
+    O = f5(s) G / ||G|| and W' = W - lr sqrt(max(1, r/c)) O."""
+    u = np.array([1.0, 2.0, 2.0]) / 3.0            # unit vectors
+    v = np.array([3.0, 4.0]) / 5.0
+    g = 2.5 * np.outer(u, v)                         # 3 x 2 (tall) or 2 x 3 (wide), ||G|| = 2.5
+    if not tall:
+        g = g.T
+    mu, eps, lr = 0.5, 0.25, 0.1
+    w = np.full(g.shape, 0.125)
+    w_new, m_new, o = oracle.muon_step_matrix(w, g.astype(np.float32), np.zeros(g.shape, np.float32), lr=lr,
+                                              mu=mu, nesterov=True, eps=eps)
+    s = (1 + mu) * 2.5 / ((1 + mu) * 2.5 + eps)
+    f5 = scalar_map(np.array([s]), [QUINTIC] * 5)[0]
+    # G is rounded to float32 on the way in; compare at float32 resolution
+    assert np.allclose(o, f5 * g / 2.5, rtol=1e-6, atol=1e-7)
+    scale = math.sqrt(max(1.0, g.shape[0] / g.shape[1]))
+    assert np.allclose(w_new, w - lr * scale * o, rtol=0, atol=1e-15)
+    assert np.array_equal(m_new, g.astype(np.float32))
