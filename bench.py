@@ -66,6 +66,11 @@ def parse():
                     help="calls per step in the end-to-end pipeline; with 1 (one call for the whole set) "
                          "the weights' download must end before the next step starts")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lerp", action="store_true", help="interpolation-form momentum (muon_step_ex)")
+    ap.add_argument("--weight-decay", type=float, default=0.0, help="decoupled weight decay (muon_step_ex)")
+    ap.add_argument("--cautious", action="store_true", help="decay only where update and weight agree in sign")
+    ap.add_argument("--normuon", action="store_true",
+                    help="NorMuon rescaling of the orthogonalised update (muon_step_ex, beta2 0.95)")
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     return ap.parse_args()
 
@@ -278,6 +283,7 @@ def main():
 
     h = mb.muon_init(local)
     stream = torch.cuda.current_stream(dev)
+    options, nstate = False, None
     if args.shard:
         from muon_newton_schulz_06_b200.sharded import ShardedMuon
         sm = ShardedMuon(W, device=dev, handle=h)
@@ -289,9 +295,17 @@ def main():
     else:
         sm = None
 
+        options = args.lerp or args.weight_decay or args.cautious or args.normuon
+        nstate = [torch.zeros(min(w.shape), device=dev) for w in W] if args.normuon else None
+
         def step(grads=G, st=None):
-            mb.muon_step(h, W, grads, M, lr=LR, momentum=MU, nesterov=True, ns_steps=NS_STEPS, eps=EPS,
-                         stream=st or stream)
+            if options:
+                mb.muon_step_ex(h, W, grads, M, lr=LR, momentum=MU, nesterov=True, ns_steps=NS_STEPS, eps=EPS,
+                                momentum_form="lerp" if args.lerp else "sgd", weight_decay=args.weight_decay,
+                                cautious=args.cautious, normuon_state=nstate, stream=st or stream)
+            else:
+                mb.muon_step(h, W, grads, M, lr=LR, momentum=MU, nesterov=True, ns_steps=NS_STEPS, eps=EPS,
+                             stream=st or stream)
 
     for _ in range(max(args.warmup, 0)):
         step()
@@ -387,6 +401,11 @@ def main():
             a, b = bounds[c]
             if args.shard:
                 step(grads, st=st)
+            elif options:
+                mb.muon_step_ex(hc[c], W[a:b], grads[a:b], M[a:b], lr=LR, momentum=MU, nesterov=True,
+                                ns_steps=NS_STEPS, eps=EPS, momentum_form="lerp" if args.lerp else "sgd",
+                                weight_decay=args.weight_decay, cautious=args.cautious,
+                                normuon_state=nstate[a:b] if nstate is not None else None, stream=st)
             else:
                 mb.muon_step(hc[c], W[a:b], grads[a:b], M[a:b], lr=LR, momentum=MU, nesterov=True,
                              ns_steps=NS_STEPS, eps=EPS, stream=st)
@@ -500,6 +519,9 @@ def main():
                                                           else ""), "matrices": len(shapes),
                        "params": int(eb["numel"]), "ns_steps": NS_STEPS,
                        "coeffs": "quintic (3.4445, -4.7750, 2.0315) every step", "lr": LR, "momentum": MU,
+                       **({"options": {"momentum_form": "lerp" if args.lerp else "sgd",
+                                       "weight_decay": args.weight_decay, "cautious": args.cautious,
+                                       "normuon": args.normuon}} if options else {}),
                        "nesterov": True, "eps": EPS,
                        "l2": "no flush: inputs larger than L2 (%.1f GB of gradients per step)" % (
                            sum(g.numel() * g.element_size() for g in G) / 1e9),
