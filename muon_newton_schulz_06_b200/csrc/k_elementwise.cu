@@ -542,6 +542,219 @@ momentum_tile_tma_kernel(const __grid_constant__ EwTiledParams p) {
   if (!ok && ct == 0) atomicExch(p.status, kDevTimeout);
 }
 
+// One weight of the update pass: W - fl32(lrs*O), then the decoupled decay where it
+// applies (every entry, or only where O and the old weight agree in sign).
+__device__ __forceinline__ float apply_elem(float w0, float o, float lrs, float lrwd, int cautious) {
+  float wn = __fsub_rn(w0, __fmul_rn(lrs, o));
+  const bool agree = (o >= 0.f && w0 >= 0.f) || (o <= 0.f && w0 <= 0.f);
+  if (lrwd != 0.f && (!cautious || agree)) wn = __fsub_rn(wn, __fmul_rn(lrwd, w0));
+  return wn;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& raw, float* v) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 f = __bfloat1622float2(h[q]);
+    v[2 * q] = f.x;
+    v[2 * q + 1] = f.y;
+  }
+}
+
+__device__ __forceinline__ uint4 f32x8_to_bf16(const float* v) {
+  uint4 raw;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) h[q] = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+  return raw;
+}
+
+constexpr size_t kApplyFlatSmem = kFlatStages * 2 * kFlatGBytes + 2 * kFlatStages * sizeof(uint64_t);
+constexpr size_t kApplyTileSmem = 1024 + kFlatStages * 2 * kFlatGBytes + 2 * kFlatStages * sizeof(uint64_t);
+
+// Bulk-copy weight update of wide matrices (bf16 weights, workspace in the caller's
+// layout): unit u covers elements [u*4096, ...) of W and of O; the structure follows
+// momentum_flat_kernel.  With NorMuon, O is first scaled by its row's factor
+// (rowsq[row_base + row], one load per 8-element chunk).
+__global__ void __launch_bounds__(kFlatThreads)
+apply_flat_kernel(const __grid_constant__ EwParams p) {
+  extern __shared__ __align__(128) uint8_t asm_[];
+  uint8_t* so = asm_;                                  // [kFlatStages][8 KB] O
+  uint8_t* sw = asm_ + kFlatStages * kFlatGBytes;      // [kFlatStages][8 KB] W, then W'
+  uint64_t* full = reinterpret_cast<uint64_t*>(asm_ + 2 * kFlatStages * kFlatGBytes);
+  uint64_t* empty = full + kFlatStages;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < kFlatStages; ++s) {
+      bar_init(&full[s], 1);
+      bar_init(&empty[s], 1);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < p.total_units; unit += gridDim.x) {
+        const EwMat& m = p.mats[find_mat(p, unit)];
+        const size_t off = (size_t)(unit - m.unit_begin) * kFlatUnit;
+        const size_t numel = (size_t)m.rows * m.cols;
+        const uint32_t cnt = (uint32_t)(numel - off < (size_t)kFlatUnit ? numel - off : (size_t)kFlatUnit);
+        if (!bar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
+        bar_arrive_tx(&full[s], cnt * 4u);
+        bulk_load(so + s * kFlatGBytes, reinterpret_cast<const __nv_bfloat16*>(m.work) + off, cnt * 2u, &full[s]);
+        bulk_load(sw + s * kFlatGBytes, reinterpret_cast<const __nv_bfloat16*>(m.param) + off, cnt * 2u, &full[s]);
+        if (++s == kFlatStages) { s = 0; ph ^= 1u; }
+      }
+      if (!ok) {
+        atomicExch(p.status, kDevTimeout);
+        const uint64_t t0 = gtimer();  // copies already issued land within microseconds
+        while (gtimer() - t0 < 1000000ull) {
+        }
+      }
+    }
+    return;
+  }
+  const int ct = tid - 32;
+  int s = 0, prev = -1;
+  uint32_t ph = 0;
+  bool ok = true;
+  for (int unit = blockIdx.x; unit < p.total_units; unit += gridDim.x) {
+    const EwMat& m = p.mats[find_mat(p, unit)];
+    const size_t off = (size_t)(unit - m.unit_begin) * kFlatUnit;
+    const size_t numel = (size_t)m.rows * m.cols;
+    const uint32_t cnt = (uint32_t)(numel - off < (size_t)kFlatUnit ? numel - off : (size_t)kFlatUnit);
+    if (!bar_wait(&full[s], ph)) { ok = false; break; }
+    const uint4* os = reinterpret_cast<const uint4*>(so + s * kFlatGBytes);
+    uint4* ws = reinterpret_cast<uint4*>(sw + s * kFlatGBytes);
+#pragma unroll
+    for (int j = 0; j < kFlatUnit / 8 / kFlatCompute; ++j) {
+      const int k = ct + j * kFlatCompute;
+      if ((uint32_t)k * 8u >= cnt) break;
+      float o[8], w[8];
+      bf16x8_to_f32(os[k], o);
+      bf16x8_to_f32(ws[k], w);
+      if (p.normuon) {
+        const float f = p.rowsq[m.row_base + (int)((off + (size_t)k * 8) / (size_t)m.cols)];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) o[q] = __fmul_rn(f, o[q]);
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) w[q] = apply_elem(w[q], o[q], m.lrs, m.lrwd, p.cautious);
+      ws[k] = f32x8_to_bf16(w);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kFlatCompute) : "memory");
+    if (ct == 0) {
+      bulk_store(reinterpret_cast<__nv_bfloat16*>(m.param) + off, sw + s * kFlatGBytes, cnt * 2u);
+      bulk_commit();
+      bulk_wait_read1();
+      if (prev >= 0) bar_arrive(&empty[prev]);
+    }
+    prev = s;
+    if (++s == kFlatStages) { s = 0; ph ^= 1u; }
+  }
+  if (ct == 0) bulk_wait_all();
+  if (!ok && ct == 0) atomicExch(p.status, kDevTimeout);
+}
+
+// TMA weight update of tall matrices (bf16 weights): unit u is the 64 x 64 tile
+// (u / tiles_c, u % tiles_c) of W; the producer loads the W tile and the matching
+// transposed tile of the workspace X through the matrix's maps (128-byte swizzle);
+// thread ct owns row ct mod 64 of the tile, columns 32*(ct/64) ..+31, reads O = X^T
+// from the transposed tile, updates W in place and one thread stores the tile.  With
+// NorMuon, O is scaled by its column's factor (rowsq[row_base + column]).
+__global__ void __launch_bounds__(kFlatThreads)
+apply_tile_tma_kernel(const __grid_constant__ EwTiledParams p) {
+  extern __shared__ uint8_t atsm_raw[];
+  uint8_t* tsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(atsm_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(tsm + kFlatStages * 2 * kFlatGBytes);
+  uint64_t* empty = full + kFlatStages;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < kFlatStages; ++s) {
+      bar_init(&full[s], 1);
+      bar_init(&empty[s], 1);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  auto w_tile = [&](int s) { return tsm + s * 2 * kFlatGBytes; };
+  auto x_tile = [&](int s) { return tsm + s * 2 * kFlatGBytes + kFlatGBytes; };
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < p.total_units; unit += gridDim.x) {
+        const int mi = find_mat(p, unit);
+        const EwMat& m = p.mats[mi];
+        const int u = unit - m.unit_begin;
+        const int r0 = (u / m.tiles_c) * kEwTile, c0 = (u % m.tiles_c) * kEwTile;
+        const CUtensorMap* maps = &p.maps[kEwMapsPerMat * mi];
+        if (!bar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
+        bar_arrive_tx(&full[s], 2 * kFlatGBytes);
+        tma_load_2d(w_tile(s), &maps[0], c0, r0, &full[s]);
+        tma_load_2d(x_tile(s), &maps[1], r0, c0, &full[s]);
+        if (++s == kFlatStages) { s = 0; ph ^= 1u; }
+      }
+      if (!ok) {
+        atomicExch(p.status, kDevTimeout);
+        const uint64_t t0 = gtimer();
+        while (gtimer() - t0 < 1000000ull) {
+        }
+      }
+    }
+    return;
+  }
+  const int ct = tid - 32;
+  const int r = ct & 63, h = ct >> 6;
+  int s = 0, prev = -1;
+  uint32_t ph = 0;
+  bool ok = true;
+  for (int unit = blockIdx.x; unit < p.total_units; unit += gridDim.x) {
+    const int mi = find_mat(p, unit);
+    const EwMat& m = p.mats[mi];
+    const int u = unit - m.unit_begin;
+    const int r0 = (u / m.tiles_c) * kEwTile, c0 = (u % m.tiles_c) * kEwTile;
+    if (!bar_wait(&full[s], ph)) { ok = false; break; }
+    uint8_t* wt = w_tile(s);
+    const uint8_t* xt = x_tile(s);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // columns 32h + 8i .. +7
+      uint4* wp = reinterpret_cast<uint4*>(wt + swz128(r, 4 * h + i));
+      float w[8], o[8];
+      bf16x8_to_f32(*wp, w);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int c = 32 * h + 8 * i + q;  // X row c, column r
+        o[q] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(xt + swz128(c, r >> 3) + ((r & 7) << 1)));
+        if (p.normuon) {
+          const float f = (c0 + c < m.cols) ? __ldg(p.rowsq + m.row_base + c0 + c) : 0.f;
+          o[q] = __fmul_rn(f, o[q]);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) w[q] = apply_elem(w[q], o[q], m.lrs, m.lrwd, p.cautious);
+      *wp = f32x8_to_bf16(w);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kFlatCompute) : "memory");
+    if (ct == 0) {
+      tma_store_2d(&p.maps[kEwMapsPerMat * mi], wt, c0, r0);
+      bulk_commit();
+      bulk_wait_read1();
+      if (prev >= 0) bar_arrive(&empty[prev]);
+    }
+    prev = s;
+    if (++s == kFlatStages) { s = 0; ph ^= 1u; }
+  }
+  if (ct == 0) bulk_wait_all();
+  if (!ok && ct == 0) atomicExch(p.status, kDevTimeout);
+}
+
 // scale[gid] = 1 / (sqrt(sum of the matrix's partials) + eps): one block per matrix,
 // fixed summation order (strided per thread, then a fixed tree), in double.
 __global__ void __launch_bounds__(kThreads)
@@ -810,6 +1023,48 @@ cudaError_t launch_momentum_split(const EwParams& flat, const EwTiledParams* til
     norm_finalize_kernel<<<all.n_mats, kThreads, 0, st>>>(all);
     ++*launches;
     return cudaGetLastError();
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_apply_split(const EwParams& flat, const EwTiledParams* tiled, int n_tiled, const EwParams& rest,
+                               int sm_count, int* launches, cudaStream_t st) {
+  *launches = 0;
+  static bool smem_set[64] = {};  // per device
+  int dev = 0;
+  cudaError_t e0 = cudaGetDevice(&dev);
+  if (e0 != cudaSuccess) return e0;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!smem_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(apply_flat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kApplyFlatSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(apply_tile_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kApplyTileSmem);
+    if (e != cudaSuccess) return e;
+    smem_set[dev] = true;
+  }
+  for (int t = 0; t < n_tiled; ++t) {
+    if (tiled[t].n_mats == 0 || tiled[t].total_units == 0) continue;
+    const int grid = std::max(1, std::min(tiled[t].total_units, 2 * sm_count));
+    apply_tile_tma_kernel<<<grid, kFlatThreads, kApplyTileSmem, st>>>(tiled[t]);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ++*launches;
+  }
+  if (flat.n_mats > 0 && flat.total_units > 0) {
+    const int grid = std::max(1, std::min(flat.total_units, 2 * sm_count));
+    apply_flat_kernel<<<grid, kFlatThreads, kApplyFlatSmem, st>>>(flat);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ++*launches;
+  }
+  if (rest.n_mats > 0 && rest.total_units > 0) {
+    const int grid = std::max(1, std::min(rest.total_units, sm_count * 8));
+    apply_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(rest, kEwApply);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ++*launches;
   }
   return cudaSuccess;
 }

@@ -98,6 +98,9 @@ struct muon_handle {
   // pointers they were encoded for (grad, momentum, workspace); cleared with the plan
   std::vector<CUtensorMap> ewmap;
   std::vector<const void*> ewmap_key;
+  // the same for the weight-update pass (weights, final workspace X)
+  std::vector<CUtensorMap> ewmap_apply;
+  std::vector<const void*> ewmap_apply_key;
   // per-launch timing (muon_profile_enable)
   bool profiling = false;
   std::vector<cudaEvent_t> ev_free;
@@ -226,6 +229,8 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
   P = Plan();
   h->ewmap.clear();  // the momentum-pass tensor maps describe the old plan's buffers
   h->ewmap_key.clear();
+  h->ewmap_apply.clear();
+  h->ewmap_apply_key.clear();
   P.mode = mode;
   const size_t esz = (mode == MUON_MODE_BF16) ? 2 : 4;
   // every per-call count below must fit the 32-bit fields of the kernels' tables
@@ -531,6 +536,88 @@ cudaError_t launch_momentum_bf16(muon_handle* h, const EwParams& ep, int b, int*
   return err;
 }
 
+// Weight-update pass of one batch in bf16 mode (bf16 weights): wide matrices whose
+// workspace copy has the caller's layout through the bulk-copy kernel, tall ones through
+// the TMA tile kernel (weight and workspace maps by value, re-encoded only when
+// pointers change), the others through the register tile kernel.
+cudaError_t launch_apply_bf16(muon_handle* h, const EwParams& ep, int b, int* launches, cudaStream_t st) {
+  const size_t n_all = h->plan.mats.size();
+  if (h->ewmap_apply.size() != n_all * 2) {
+    h->ewmap_apply.assign(n_all * 2, CUtensorMap{});
+    h->ewmap_apply_key.assign(n_all * 2, nullptr);
+  }
+  EwParams* flat = new EwParams(ep);
+  EwParams* rest = new EwParams(ep);
+  const int max_tiled = (ep.n_mats + kMaxTiledPerLaunch - 1) / kMaxTiledPerLaunch;
+  EwTiledParams* tiled = new EwTiledParams[max_tiled > 0 ? max_tiled : 1]();
+  int n_tiled = 0;
+  flat->n_mats = rest->n_mats = 0;
+  int uf = 0, ur = 0;
+  cudaError_t err = cudaSuccess;
+  for (int j = 0; j < ep.n_mats; ++j) {
+    const EwMat& m = ep.mats[j];
+    const int i = b + j;
+    const bool aligned = (reinterpret_cast<uintptr_t>(m.param) % 16 == 0) &&
+                         (reinterpret_cast<uintptr_t>(m.work) % 16 == 0);
+    const bool eligible = m.param_bf16 && m.cols % 8 == 0 && aligned;
+    EwMat e = m;
+    if (eligible && !m.transposed && m.ld == m.cols) {
+      const int64_t numel = (int64_t)m.rows * m.cols;
+      e.n_units = (int32_t)((numel + kFlatUnit - 1) / kFlatUnit);
+      e.unit_begin = uf;
+      uf += e.n_units;
+      flat->mats[flat->n_mats++] = e;
+    } else if (eligible && m.transposed) {
+      const void** key = h->ewmap_apply_key.data() + (size_t)i * 2;
+      CUtensorMap* maps = h->ewmap_apply.data() + (size_t)i * 2;
+      if (key[0] != m.param || key[1] != m.work) {
+        const cuuint32_t estr[2] = {1, 1};
+        const cuuint32_t box[2] = {(cuuint32_t)kEwTile, (cuuint32_t)kEwTile};
+        const cuuint64_t wdims[2] = {(cuuint64_t)m.cols, (cuuint64_t)m.rows};
+        const cuuint64_t wstr[1] = {(cuuint64_t)m.cols * 2};
+        const cuuint64_t xdims[2] = {(cuuint64_t)m.rows, (cuuint64_t)m.cols};
+        const cuuint64_t xstr[1] = {(cuuint64_t)m.ld * 2};
+        CUresult r = h->encode(&maps[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, m.param, wdims, wstr, box, estr,
+                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r == CUDA_SUCCESS)
+          r = h->encode(&maps[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, m.work, xdims, xstr, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+          err = cudaErrorInvalidValue;
+          break;
+        }
+        key[0] = m.param;
+        key[1] = m.work;
+      }
+      if (n_tiled == 0 || tiled[n_tiled - 1].n_mats == kMaxTiledPerLaunch) {
+        EwTiledParams& tp = tiled[n_tiled++];
+        tp.status = ep.status;
+        tp.cautious = ep.cautious;
+        tp.normuon = ep.normuon;
+        tp.rowsq = ep.rowsq;
+      }
+      EwTiledParams& tp = tiled[n_tiled - 1];
+      std::memcpy(&tp.maps[tp.n_mats * kEwMapsPerMat], maps, 2 * sizeof(CUtensorMap));
+      e.unit_begin = tp.total_units;
+      tp.total_units += e.n_units;
+      tp.mats[tp.n_mats++] = e;
+    } else {
+      e.unit_begin = ur;
+      ur += e.n_units;
+      rest->mats[rest->n_mats++] = e;
+    }
+  }
+  flat->total_units = uf;
+  rest->total_units = ur;
+  if (err == cudaSuccess) err = launch_apply_split(*flat, tiled, n_tiled, *rest, h->sm_count, launches, st);
+  delete flat;
+  delete rest;
+  delete[] tiled;
+  return err;
+}
+
 muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, int pass, int out_kind,
                                int work_buf, const CallOpts& o, cudaStream_t st) {
   const bool momentum_pass = pass == kPassMomentum;
@@ -594,6 +681,8 @@ muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, i
     cudaError_t err;
     if (pass == kPassMomentum && ep->use_momentum && !f32) {
       err = launch_momentum_bf16(h, *ep, b, &launches, st);
+    } else if (pass == kPassOut && out_kind == kEwApply && !f32) {
+      err = launch_apply_bf16(h, *ep, b, &launches, st);
     } else {
       err = pass == kPassMomentum ? launch_momentum_norm(*ep, f32, grid, st)
             : pass == kPassNormuon ? launch_normuon(*ep, f32, h->sm_count * 8, st)

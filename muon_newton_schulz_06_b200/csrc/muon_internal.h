@@ -88,6 +88,10 @@ struct __align__(64) EwTiledParams {
   float omu;
   float* partials;
   int* status;
+  // apply pass of tall matrices (maps per matrix: weights, final workspace X)
+  int cautious;
+  int normuon;
+  const float* rowsq;   // NorMuon per-row factors (indexed by row_base + caller column)
 };
 static_assert(sizeof(EwTiledParams) <= 32764, "tiled momentum parameters must fit the kernel parameter space");
 
@@ -109,6 +113,11 @@ cudaError_t launch_momentum_norm(const EwParams& p, bool work_f32, int grid, cud
 cudaError_t launch_momentum_split(const EwParams& flat, const EwTiledParams* tiled, int n_tiled, const EwParams& rest,
                                   const EwParams& all, int sm_count, int* launches, cudaStream_t st);
 cudaError_t launch_apply(const EwParams& p, bool work_f32, int out_kind, int grid, cudaStream_t st);
+// Weight-update pass split like the momentum pass (bf16 weights and workspace): `flat`
+// wide matrices through bulk copies, `tiled[0..n_tiled)` tall ones through tensor maps
+// (maps[0] = weights, maps[1] = workspace X), `rest` through the register tile kernel.
+cudaError_t launch_apply_split(const EwParams& flat, const EwTiledParams* tiled, int n_tiled, const EwParams& rest,
+                               int sm_count, int* launches, cudaStream_t st);
 
 // ----------------------------------------------------------------- tensor-core engine
 
