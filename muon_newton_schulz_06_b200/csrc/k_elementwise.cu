@@ -569,19 +569,22 @@ __device__ __forceinline__ uint4 f32x8_to_bf16(const float* v) {
   return raw;
 }
 
-constexpr size_t kApplyFlatSmem = kFlatStages * 2 * kFlatGBytes + 2 * kFlatStages * sizeof(uint64_t);
+// The weight update moves half the bytes per element of the momentum pass, so its bulk
+// units are twice as long (8192 elements, 16 KB of O and 16 KB of W per stage).
+constexpr uint32_t kApplyStageBytes = kApplyUnit * 2;  // one bf16 operand of a unit
+constexpr size_t kApplyFlatSmem = kFlatStages * 2 * kApplyStageBytes + 2 * kFlatStages * sizeof(uint64_t);
 constexpr size_t kApplyTileSmem = 1024 + kFlatStages * 2 * kFlatGBytes + 2 * kFlatStages * sizeof(uint64_t);
 
 // Bulk-copy weight update of wide matrices (bf16 weights, workspace in the caller's
-// layout): unit u covers elements [u*4096, ...) of W and of O; the structure follows
+// layout): unit u covers elements [u*8192, ...) of W and of O; the structure follows
 // momentum_flat_kernel.  With NorMuon, O is first scaled by its row's factor
 // (rowsq[row_base + row], one load per 8-element chunk).
 __global__ void __launch_bounds__(kFlatThreads)
 apply_flat_kernel(const __grid_constant__ EwParams p) {
   extern __shared__ __align__(128) uint8_t asm_[];
-  uint8_t* so = asm_;                                  // [kFlatStages][8 KB] O
-  uint8_t* sw = asm_ + kFlatStages * kFlatGBytes;      // [kFlatStages][8 KB] W, then W'
-  uint64_t* full = reinterpret_cast<uint64_t*>(asm_ + 2 * kFlatStages * kFlatGBytes);
+  uint8_t* so = asm_;                                       // [kFlatStages][16 KB] O
+  uint8_t* sw = asm_ + kFlatStages * kApplyStageBytes;      // [kFlatStages][16 KB] W, then W'
+  uint64_t* full = reinterpret_cast<uint64_t*>(asm_ + 2 * kFlatStages * kApplyStageBytes);
   uint64_t* empty = full + kFlatStages;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
@@ -599,13 +602,13 @@ apply_flat_kernel(const __grid_constant__ EwParams p) {
       bool ok = true;
       for (int unit = blockIdx.x; unit < p.total_units; unit += gridDim.x) {
         const EwMat& m = p.mats[find_mat(p, unit)];
-        const size_t off = (size_t)(unit - m.unit_begin) * kFlatUnit;
+        const size_t off = (size_t)(unit - m.unit_begin) * kApplyUnit;
         const size_t numel = (size_t)m.rows * m.cols;
-        const uint32_t cnt = (uint32_t)(numel - off < (size_t)kFlatUnit ? numel - off : (size_t)kFlatUnit);
+        const uint32_t cnt = (uint32_t)(numel - off < (size_t)kApplyUnit ? numel - off : (size_t)kApplyUnit);
         if (!bar_wait(&empty[s], ph ^ 1u)) { ok = false; break; }
         bar_arrive_tx(&full[s], cnt * 4u);
-        bulk_load(so + s * kFlatGBytes, reinterpret_cast<const __nv_bfloat16*>(m.work) + off, cnt * 2u, &full[s]);
-        bulk_load(sw + s * kFlatGBytes, reinterpret_cast<const __nv_bfloat16*>(m.param) + off, cnt * 2u, &full[s]);
+        bulk_load(so + s * kApplyStageBytes, reinterpret_cast<const __nv_bfloat16*>(m.work) + off, cnt * 2u, &full[s]);
+        bulk_load(sw + s * kApplyStageBytes, reinterpret_cast<const __nv_bfloat16*>(m.param) + off, cnt * 2u, &full[s]);
         if (++s == kFlatStages) { s = 0; ph ^= 1u; }
       }
       if (!ok) {
@@ -623,23 +626,33 @@ apply_flat_kernel(const __grid_constant__ EwParams p) {
   bool ok = true;
   for (int unit = blockIdx.x; unit < p.total_units; unit += gridDim.x) {
     const EwMat& m = p.mats[find_mat(p, unit)];
-    const size_t off = (size_t)(unit - m.unit_begin) * kFlatUnit;
+    const size_t off = (size_t)(unit - m.unit_begin) * kApplyUnit;
     const size_t numel = (size_t)m.rows * m.cols;
-    const uint32_t cnt = (uint32_t)(numel - off < (size_t)kFlatUnit ? numel - off : (size_t)kFlatUnit);
-    if (!bar_wait(&full[s], ph)) { ok = false; break; }
-    const uint4* os = reinterpret_cast<const uint4*>(so + s * kFlatGBytes);
-    uint4* ws = reinterpret_cast<uint4*>(sw + s * kFlatGBytes);
+    const uint32_t cnt = (uint32_t)(numel - off < (size_t)kApplyUnit ? numel - off : (size_t)kApplyUnit);
+    float fac[kApplyUnit / 8 / kFlatCompute];  // NorMuon factor of each chunk's row (read while
+    if (p.normuon) {                           // the unit's copies are still landing)
+      const size_t r_first = off / (size_t)m.cols;  // row of the unit's first element
+      const uint32_t rem = (uint32_t)(off - r_first * (size_t)m.cols);
 #pragma unroll
-    for (int j = 0; j < kFlatUnit / 8 / kFlatCompute; ++j) {
+      for (int j = 0; j < kApplyUnit / 8 / kFlatCompute; ++j) {
+        const uint32_t k = (uint32_t)(ct + j * kFlatCompute);
+        fac[j] = k * 8u < cnt ? __ldg(p.rowsq + m.row_base + (int)(r_first + (rem + 8u * k) / (uint32_t)m.cols))
+                              : 0.f;
+      }
+    }
+    if (!bar_wait(&full[s], ph)) { ok = false; break; }
+    const uint4* os = reinterpret_cast<const uint4*>(so + s * kApplyStageBytes);
+    uint4* ws = reinterpret_cast<uint4*>(sw + s * kApplyStageBytes);
+#pragma unroll
+    for (int j = 0; j < kApplyUnit / 8 / kFlatCompute; ++j) {
       const int k = ct + j * kFlatCompute;
       if ((uint32_t)k * 8u >= cnt) break;
       float o[8], w[8];
       bf16x8_to_f32(os[k], o);
       bf16x8_to_f32(ws[k], w);
       if (p.normuon) {
-        const float f = p.rowsq[m.row_base + (int)((off + (size_t)k * 8) / (size_t)m.cols)];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) o[q] = __fmul_rn(f, o[q]);
+        for (int q = 0; q < 8; ++q) o[q] = __fmul_rn(fac[j], o[q]);
       }
 #pragma unroll
       for (int q = 0; q < 8; ++q) w[q] = apply_elem(w[q], o[q], m.lrs, m.lrwd, p.cautious);
@@ -648,7 +661,7 @@ apply_flat_kernel(const __grid_constant__ EwParams p) {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("bar.sync 1, %0;" ::"n"(kFlatCompute) : "memory");
     if (ct == 0) {
-      bulk_store(reinterpret_cast<__nv_bfloat16*>(m.param) + off, sw + s * kFlatGBytes, cnt * 2u);
+      bulk_store(reinterpret_cast<__nv_bfloat16*>(m.param) + off, sw + s * kApplyStageBytes, cnt * 2u);
       bulk_commit();
       bulk_wait_read1();
       if (prev >= 0) bar_arrive(&empty[prev]);
@@ -719,6 +732,10 @@ apply_tile_tma_kernel(const __grid_constant__ EwTiledParams p) {
     const EwMat& m = p.mats[mi];
     const int u = unit - m.unit_begin;
     const int r0 = (u / m.tiles_c) * kEwTile, c0 = (u % m.tiles_c) * kEwTile;
+    // NorMuon factor of column 32h + lane (all lanes of a warp share h), broadcast below;
+    // read while the tile's copies are still landing
+    float fac_lane = 0.f;
+    if (p.normuon && c0 + 32 * h + lane < m.cols) fac_lane = __ldg(p.rowsq + m.row_base + c0 + 32 * h + lane);
     if (!bar_wait(&full[s], ph)) { ok = false; break; }
     uint8_t* wt = w_tile(s);
     const uint8_t* xt = x_tile(s);
@@ -731,10 +748,7 @@ apply_tile_tma_kernel(const __grid_constant__ EwTiledParams p) {
       for (int q = 0; q < 8; ++q) {
         const int c = 32 * h + 8 * i + q;  // X row c, column r
         o[q] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(xt + swz128(c, r >> 3) + ((r & 7) << 1)));
-        if (p.normuon) {
-          const float f = (c0 + c < m.cols) ? __ldg(p.rowsq + m.row_base + c0 + c) : 0.f;
-          o[q] = __fmul_rn(f, o[q]);
-        }
+        if (p.normuon) o[q] = __fmul_rn(__shfl_sync(0xffffffffu, fac_lane, 8 * i + q), o[q]);
       }
 #pragma unroll
       for (int q = 0; q < 8; ++q) w[q] = apply_elem(w[q], o[q], m.lrs, m.lrwd, p.cautious);

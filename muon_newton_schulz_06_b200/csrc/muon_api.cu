@@ -563,7 +563,7 @@ cudaError_t launch_apply_bf16(muon_handle* h, const EwParams& ep, int b, int* la
     EwMat e = m;
     if (eligible && !m.transposed && m.ld == m.cols) {
       const int64_t numel = (int64_t)m.rows * m.cols;
-      e.n_units = (int32_t)((numel + kFlatUnit - 1) / kFlatUnit);
+      e.n_units = (int32_t)((numel + kApplyUnit - 1) / kApplyUnit);
       e.unit_begin = uf;
       uf += e.n_units;
       flat->mats[flat->n_mats++] = e;

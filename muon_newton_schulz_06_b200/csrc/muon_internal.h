@@ -28,6 +28,8 @@ constexpr int kWarpsPerUnit = 8;
 // as many elements as a 64 x 64 tile, so a matrix never has more of these units than
 // tiles and the partials array sized for tiles holds them.
 constexpr int kFlatUnit = kEwTile * kEwTile;
+// Unit of the bulk-copy weight-update pass (no partials, so not tied to the tile count).
+constexpr int kApplyUnit = 2 * kFlatUnit;
 
 struct EwMat {
   void* param;          // caller matrix: param (apply), or x_in (normalise-only)
