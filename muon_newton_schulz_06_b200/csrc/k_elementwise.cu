@@ -18,14 +18,15 @@
 // partial sum (fixed shuffle tree), and a second small kernel adds a matrix's partials
 // in a fixed order.
 //
-// In bf16 mode the momentum pass moves data with the copy engine instead: wide matrices
-// (workspace copy in the caller's layout) in units of 4096 contiguous elements through
-// cp.async.bulk, tall ones in 64 x 64 tiles through tensor maps (cp.async.bulk.tensor,
-// 128-byte swizzle, transposed in shared memory), each through a 3-stage ring per CTA.
-// The bytes in flight are then bounded by shared memory rather than by registers, and
-// the pass keeps HBM busy at the reduced SM clock of a power-capped step (the register
-// tile kernel is bound by load latency there).  Matrices that fit neither (fp32
-// gradients, unaligned rows) keep the register tile kernel.
+// In bf16 mode the momentum pass and the weight update move data with the copy engine
+// instead: wide matrices (workspace copy in the caller's layout) in contiguous units
+// through cp.async.bulk (4096 elements for the momentum pass, 8192 for the update), tall
+// ones in 64 x 64 tiles through tensor maps (cp.async.bulk.tensor, 128-byte swizzle,
+// transposed in shared memory), each through a 3-stage ring per CTA.  The bytes in
+// flight are then bounded by shared memory rather than by registers, and the passes
+// keep HBM busy at the reduced SM clock of a power-capped step (the register tile
+// kernels are bound by load latency there).  Matrices that fit neither (fp32 gradients
+// or weights, unaligned rows) keep the register tile kernels.
 #include <algorithm>
 
 #include "muon_internal.h"
@@ -35,7 +36,7 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// ---- bulk-copy helpers (momentum_flat_kernel)
+// ---- copy-engine helpers (bulk-copy and tensor-map kernels)
 __device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 __device__ __forceinline__ uint64_t gtimer() {
   uint64_t t;
