@@ -38,7 +38,11 @@
  *    cudaMalloc, on the first call with a new list of shapes and mode, and reused
  *    by later calls with the same list; such calls allocate nothing.  Calls that
  *    share a handle must not overlap on the GPU (use one stream per handle, or
- *    one handle per stream).  A handle is not thread-safe.
+ *    one handle per stream).  A handle is not thread-safe; distinct handles may be
+ *    used from distinct host threads.
+ *  - With the environment variable MUON_LOG set (and not "0") when a handle is
+ *    created, that handle writes its plans (shape groups, tile counts, workspace
+ *    bytes) and the detail of every error to stderr.
  */
 #ifndef MUON_B200_MUON_H
 #define MUON_B200_MUON_H
@@ -180,10 +184,14 @@ MUON_API muon_status muon_newton_schulz(muon_handle_t h, const void* const* x_in
  * cudaFree or other allocating routine.
  *
  * Computes what muon_newton_schulz computes in MUON_MODE_BF16 for a single matrix,
- * with the same kernels: o_out = Newton-Schulz of x_in / (||x_in||_F + eps).
+ * with the same kernels in the same order (norm pass, tensor-core steps, export), so
+ * the two give the same bits: o_out = Newton-Schulz of x_in / (||x_in||_F + eps).
+ * A call enqueues kernels and a 4-byte memset only; it makes no host-to-device copy.
  *  x_in, o_out   DEVICE pointers on the CURRENT device, rows x cols of `dtype`,
- *                row-major, 16-byte aligned, not overlapping; caller-owned
- *  status        optional DEVICE int (4-byte aligned); if not NULL, a bounded wait
+ *                row-major, 16-byte aligned, not overlapping; caller-owned.  A
+ *                pointer that is not device memory of the current device (host
+ *                memory, another GPU's memory) returns MUON_ERR_INVALID_ARG
+ *  status        optional DEVICE int (4-byte aligned, current device); if not NULL, a bounded wait
  *                that expires inside a kernel stores 1 there (the caller clears it);
  *                if NULL, such a time-out goes unreported
  *  coeffs, ns_steps, eps, cuda_stream   as in muon_newton_schulz
@@ -215,6 +223,14 @@ MUON_API muon_status muon_sync(muon_handle_t h);
  * MUON_ERR_TIMEOUT (and clears).  The GPU context stays usable.  Returns
  * MUON_ERR_INVALID_ARG for a NULL handle or a limit out of range. */
 MUON_API muon_status muon_selftest_wait_timeout(muon_handle_t h, int64_t limit_ns, void* cuda_stream);
+
+/* Diagnostic for the allocation-failure path: the next time the handle must allocate
+ * its workspace (a call with a new list of shapes or mode that needs more than the
+ * handle holds), the allocation reports failure as if cudaMalloc had failed, once.
+ * That call returns MUON_ERR_OOM with nothing enqueued, the handle then holds no
+ * workspace, and the next call allocates normally.  No device work.  Returns
+ * MUON_ERR_INVALID_ARG for a NULL handle. */
+MUON_API muon_status muon_selftest_fail_next_alloc(muon_handle_t h);
 
 /* Bytes of device workspace the handle currently holds. */
 MUON_API int64_t muon_workspace_bytes(muon_handle_t h);

@@ -34,7 +34,7 @@ MUON_MODE_FP32_VALIDATE = 1
 
 EXPORTED = ("muon_init", "muon_step", "muon_step_ex", "muon_newton_schulz", "muon_newton_schulz_noalloc",
             "muon_sync",
-            "muon_selftest_wait_timeout", "muon_workspace_bytes",
+            "muon_selftest_wait_timeout", "muon_selftest_fail_next_alloc", "muon_workspace_bytes",
             "muon_last_launch_count", "muon_profile_enable", "muon_profile_read", "muon_destroy",
             "muon_status_string", "muon_last_error")
 
@@ -93,6 +93,8 @@ def load_library(path: str = LIB_PATH):
     lib.muon_newton_schulz_noalloc.restype = i32
     lib.muon_selftest_wait_timeout.argtypes = [vp, i64, vp]
     lib.muon_selftest_wait_timeout.restype = i32
+    lib.muon_selftest_fail_next_alloc.argtypes = [vp]
+    lib.muon_selftest_fail_next_alloc.restype = i32
     lib.muon_sync.argtypes = [vp]
     lib.muon_sync.restype = i32
     lib.muon_workspace_bytes.argtypes = [vp]
@@ -271,21 +273,33 @@ def muon_newton_schulz_noalloc(x: torch.Tensor, out: torch.Tensor, coeffs=None, 
     _check_tensor(out, "out")
     if _dtype_code(x) != _dtype_code(out) or out.shape != x.shape:
         raise ValueError("x and out must share shape and dtype")
+    if out.device != x.device:
+        raise ValueError("x and out must be on the same device")
     st_ptr = None
     if status is not None:
         if not status.is_cuda or status.dtype != torch.int32:
             raise TypeError("status must be an int32 CUDA tensor")
+        if status.device != x.device:
+            raise ValueError("status must be on the device of x")
         st_ptr = status.data_ptr()
     c = _coeff_array(coeffs, ns_steps)
-    _check(load_library().muon_newton_schulz_noalloc(x.data_ptr(), out.data_ptr(), x.shape[0], x.shape[1],
-                                                     _dtype_code(x), c, int(ns_steps), float(eps), st_ptr,
-                                                     _stream_ptr(stream, x.device)))
+    # the library works on the current device: make it x's for the call
+    with torch.cuda.device(x.device):
+        _check(load_library().muon_newton_schulz_noalloc(x.data_ptr(), out.data_ptr(), x.shape[0], x.shape[1],
+                                                         _dtype_code(x), c, int(ns_steps), float(eps), st_ptr,
+                                                         _stream_ptr(stream, x.device)))
 
 
 def muon_selftest_wait_timeout(handle, limit_ns: int, stream=None) -> None:
     """Enqueues the bounded-wait diagnostic (see include/muon.h); the next muon_sync
     raises MuonError with code MUON_ERR_TIMEOUT."""
     _check(load_library().muon_selftest_wait_timeout(handle, int(limit_ns), _stream_ptr(stream, None)), handle)
+
+
+def muon_selftest_fail_next_alloc(handle) -> None:
+    """Makes the handle's next workspace allocation report failure once (see
+    include/muon.h); that call raises MuonError with code MUON_ERR_OOM."""
+    _check(load_library().muon_selftest_fail_next_alloc(handle), handle)
 
 
 def muon_sync(handle) -> None:

@@ -34,6 +34,9 @@
 // of tile t+1.  Every mbarrier wait is bounded in time; on expiry the kernel writes
 // kDevTimeout to the status word, tells the peer CTA, lets its own copies and MMAs
 // drain, frees TMEM and returns.
+#include <atomic>
+#include <mutex>
+
 #include "muon_internal.h"
 
 namespace muon {
@@ -748,17 +751,23 @@ cudaError_t set_smem_attr() {
 }
 
 struct DeviceInfo {
-  bool ready = false;
+  std::atomic<bool> ready{false};
   int clusters = 0;
 };
 DeviceInfo g_dev_info[64];
+// Serialises the first set-up of a device between host threads (several handles, or
+// the allocation-free entry point, may reach it at once); later calls only read
+// `ready` (acquire) and the values published before it.
+std::mutex g_dev_setup_mutex;
 
 // Sets the shared-memory attribute of every phase on the current device and finds how
 // many 2-CTA clusters of this kernel fit at once.
 cudaError_t device_setup(int dev) {
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   DeviceInfo& d = g_dev_info[dev];
-  if (d.ready) return cudaSuccess;
+  if (d.ready.load(std::memory_order_acquire)) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(g_dev_setup_mutex);
+  if (d.ready.load(std::memory_order_relaxed)) return cudaSuccess;
   cudaError_t e = set_smem_attr<kPhaseGram, TcNoApply>();
   if (e == cudaSuccess) e = set_smem_attr<kPhasePoly, TcNoApply>();
   if (e == cudaSuccess) e = set_smem_attr<kPhaseUpdate, TcNoApply>();
@@ -785,7 +794,7 @@ cudaError_t device_setup(int dev) {
     n = sms / 2;
   }
   d.clusters = n;
-  d.ready = true;
+  d.ready.store(true, std::memory_order_release);
   return cudaSuccess;
 }
 

@@ -15,6 +15,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -112,6 +113,10 @@ struct muon_handle {
   cudaEvent_t ev_open = nullptr;
   double prof_ms[MUON_KIND_COUNT] = {};
   int64_t prof_launches[MUON_KIND_COUNT] = {};
+  // muon_selftest_fail_next_alloc: the next workspace allocation reports failure
+  bool fail_next_alloc = false;
+  // MUON_LOG set (and not "0") at muon_init: plan summaries and errors go to stderr
+  bool log = false;
 };
 
 namespace {
@@ -124,6 +129,7 @@ muon_status fail(muon_handle* h, muon_status st, const char* fmt, ...) {
     vsnprintf(buf, sizeof(buf), fmt, ap);
     va_end(ap);
     h->err = buf;
+    if (h->log) fprintf(stderr, "muon: %s: %s\n", muon_status_string(st), buf);
   }
   return st;
 }
@@ -343,9 +349,12 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
       h->ws_bytes = 0;
     }
     void* p = nullptr;
-    if (cudaMalloc(&p, P.bytes) != cudaSuccess) {
+    const bool injected = h->fail_next_alloc;
+    h->fail_next_alloc = false;
+    if (injected || cudaMalloc(&p, P.bytes) != cudaSuccess) {
       cudaGetLastError();
-      return fail(h, MUON_ERR_OOM, "workspace allocation of %zu bytes failed", P.bytes);
+      return fail(h, MUON_ERR_OOM, "workspace allocation of %zu bytes failed%s", P.bytes,
+                  injected ? " (injected by muon_selftest_fail_next_alloc)" : "");
     }
     h->ws = static_cast<char*>(p);
     h->ws_bytes = P.bytes;
@@ -390,6 +399,17 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
     }
   }
   P.valid = true;
+  if (h->log) {
+    size_t n_tiles[3] = {0, 0, 0};
+    for (const ChunkPlan& c : P.chunks)
+      for (int ph = 0; ph < 3; ++ph) n_tiles[ph] += (size_t)c.n_tiles[ph];
+    fprintf(stderr,
+            "muon: plan: %d matrices, %zu shape groups, %zu launch chunks, tiles gram/poly/update %zu/%zu/%zu, "
+            "workspace %zu bytes (%s mode)\n",
+            n, P.groups.size(), P.chunks.size(), n_tiles[0], n_tiles[1], n_tiles[2], P.bytes,
+            mode == MUON_MODE_BF16 ? "bf16" : "fp32");
+    for (const GroupPlan& g : P.groups) fprintf(stderr, "muon:   group s=%d L=%d n=%d\n", g.s, g.L, g.n);
+  }
   return MUON_OK;
 }
 
@@ -921,6 +941,9 @@ muon_status muon_init(muon_handle_t* out, int device) {
   h->device = device;
   h->sm_count = prop.multiProcessorCount;
   h->encode = reinterpret_cast<EncodeTiledFn>(fn);
+  const char* lg = getenv("MUON_LOG");
+  h->log = lg != nullptr && lg[0] != '\0' && strcmp(lg, "0") != 0;
+  if (h->log) fprintf(stderr, "muon: handle on device %d (%s, %d SMs)\n", device, prop.name, h->sm_count);
   *out = h;
   return MUON_OK;
 }
@@ -1084,6 +1107,12 @@ muon_status muon_selftest_wait_timeout(muon_handle_t h, int64_t limit_ns, void* 
   if (e != cudaSuccess) return cuda_fail(h, e, "self-test launch");
   h->last_launches = 1;
   return finish_call(h, st);
+}
+
+muon_status muon_selftest_fail_next_alloc(muon_handle_t h) {
+  if (!h) return MUON_ERR_INVALID_ARG;
+  h->fail_next_alloc = true;
+  return MUON_OK;
 }
 
 muon_status muon_sync(muon_handle_t h) {

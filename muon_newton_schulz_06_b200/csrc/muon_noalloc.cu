@@ -16,10 +16,12 @@
 // cudaGetSymbolAddress and caches it.  Every call shares the array and leaves its
 // contents behind, so each call re-zeroes what must start at zero (the internal status
 // word; every other region is fully written before it is read), and calls that overlap
-// on the GPU race.
+// on the GPU race.  The tile lists are written into the array by a small kernel on the
+// caller's stream, so a call makes no host-to-device copy.
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "muon.h"
 #include "muon_internal.h"
@@ -29,7 +31,7 @@ using namespace muon;
 namespace {
 
 constexpr size_t kScratchBytes = size_t(32) << 20;  // 32 MiB per device
-constexpr int kMaxTiles = 16384;                     // entries of the host tile staging area
+constexpr int kMaxTiles = 16384;                     // tile-list entries kept in the scratch
 constexpr int kMaxDevices = 64;
 constexpr float kDefaultTriple[3] = {3.4445f, -4.7750f, 2.0315f};
 
@@ -43,11 +45,43 @@ typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void
 // the first call on that device), the tensor-map encoder, and the parameter blocks.
 char* g_scratch_addr[kMaxDevices] = {};
 EncodeFn g_encode = nullptr;
-TcTile g_tiles[kMaxTiles];
 EwParams g_ew;
 TcParams g_tc;
 
+std::mutex g_setup_mutex;  // first call on a device from several host threads
+
 size_t up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Tile lists of one s x L (wide orientation) matrix, in the order of tc_syrk_tiles and
+// tc_update_tiles: entries [0, n_syrk) are the 256 x 256 blocks (bi <= bj) of the
+// symmetric products, row-block major; entries [n_syrk, n_syrk + n_upd) the blocks of
+// the update, column-block major.  One thread per entry.
+__global__ void noalloc_tiles_kernel(TcTile* out, int s, int L, int n_syrk, int n_upd) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= n_syrk + n_upd) return;
+  const int nb = (s + kTile - 1) / kTile;
+  if (t < n_syrk) {
+    int bi = 0, first = 0;  // first = index of tile (bi, bi)
+    while (first + (nb - bi) <= t) {
+      first += nb - bi;
+      ++bi;
+    }
+    out[t] = TcTile{0, 0, (uint16_t)bi, (uint16_t)(bi + (t - first))};
+  } else {
+    const int u = t - n_syrk, mb = nb;
+    out[t] = TcTile{0, 0, (uint16_t)(u % mb), (uint16_t)(u / mb)};
+  }
+}
+
+// True when p is device memory of device `dev` (plain or managed allocation).
+bool on_device(const void* p, int dev) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) && a.device == dev;
+}
 
 bool encode(CUtensorMap* map, void* base, int inner, int rows, int ld, int box_inner, int box_rows,
             CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
@@ -105,7 +139,10 @@ extern "C" MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, voi
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MUON_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return MUON_ERR_UNSUPPORTED;
+  if (!on_device(x_in, dev) || !on_device(o_out, dev) || (status && !on_device(status, dev)))
+    return MUON_ERR_INVALID_ARG;
   if (!g_scratch_addr[dev]) {
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
@@ -119,6 +156,7 @@ extern "C" MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, voi
     g_scratch_addr[dev] = static_cast<char*>(p);
   }
   if (!g_encode) {
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
@@ -132,11 +170,10 @@ extern "C" MUON_API muon_status muon_newton_schulz_noalloc(const void* x_in, voi
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
 
   // ---- tile lists (Gram and Poly share the triangle list) and zeroed words
-  const int t = tc_syrk_tiles(s, 0, 0, g_tiles) + tc_update_tiles(s, L, 0, 0, g_tiles + n_syrk);
-  // pageable source: the copy is staged before the call returns, so g_tiles may be reused
-  if (cudaMemcpyAsync(scr + off_tiles, g_tiles, (size_t)t * sizeof(TcTile), cudaMemcpyHostToDevice, st) !=
-      cudaSuccess)
-    return MUON_ERR_CUDA;
+  const int n_tiles = n_syrk + n_upd;
+  noalloc_tiles_kernel<<<(n_tiles + 255) / 256, 256, 0, st>>>(reinterpret_cast<TcTile*>(scr + off_tiles), s, L,
+                                                             n_syrk, n_upd);
+  if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   if (cudaMemsetAsync(scr + off_status, 0, 4, st) != cudaSuccess) return MUON_ERR_CUDA;
   int* stat = status ? status : reinterpret_cast<int*>(scr + off_status);
 

@@ -1,4 +1,4 @@
-"""Failure detection without a GPU fault.
+"""Failure detection without a GPU fault, and the hygiene paths around it.
 
 The library bounds every device-side wait; when one expires, the kernel records a
 time-out in the handle's status word and returns, and the host reports
@@ -72,3 +72,112 @@ def test_selftest_rejects_bad_limits(mb):
         assert e.value.code == mb.MUON_ERR_INVALID_ARG
     finally:
         mb.muon_destroy(h)
+
+
+# ---------------------------------------------------------------- allocation failure (injected on the host)
+
+def test_injected_allocation_failure_leaves_the_handle_usable(mb):
+    """The workspace allocation is made to fail on the host (no device fault): the call
+    returns MUON_ERR_OOM with nothing enqueued, and the next call allocates and runs."""
+    h = mb.muon_init(0)
+    try:
+        w = torch.zeros(64, 32, device="cuda")
+        g = torch.randn(64, 32, device="cuda")
+        m = torch.zeros(64, 32, device="cuda")
+        mb.muon_selftest_fail_next_alloc(h)
+        with pytest.raises(mb.MuonError) as e:
+            mb.muon_step(h, [w], [g], [m], lr=1.0)
+        assert e.value.code == mb.MUON_ERR_OOM
+        assert "injected" in str(e.value)
+        torch.cuda.synchronize()
+        assert torch.count_nonzero(m) == 0 and torch.count_nonzero(w) == 0
+        assert mb.muon_workspace_bytes(h) == 0
+        mb.muon_step(h, [w], [g], [m], lr=1.0)
+        torch.cuda.synchronize()
+        mb.muon_sync(h)
+        assert torch.equal(m, g) and torch.count_nonzero(w) > 0
+        held = mb.muon_workspace_bytes(h)
+        assert held > 0
+        # a handle that holds a workspace and must grow it: the old one is released first
+        W = [torch.zeros(512, 256, device="cuda") for _ in range(3)]
+        G = [torch.randn(512, 256, device="cuda") for _ in range(3)]
+        M = [torch.zeros(512, 256, device="cuda") for _ in range(3)]
+        mb.muon_selftest_fail_next_alloc(h)
+        with pytest.raises(mb.MuonError) as e:
+            mb.muon_step(h, W, G, M, lr=1.0)
+        assert e.value.code == mb.MUON_ERR_OOM
+        assert mb.muon_workspace_bytes(h) == 0
+        torch.cuda.synchronize()
+        assert all(torch.count_nonzero(x) == 0 for x in M)
+        mb.muon_step(h, W, G, M, lr=1.0)
+        torch.cuda.synchronize()
+        mb.muon_sync(h)
+        assert all(torch.equal(a, b) for a, b in zip(M, G))
+        assert mb.muon_workspace_bytes(h) > held
+    finally:
+        mb.muon_destroy(h)
+
+
+# ---------------------------------------------------------------- checkpoint / resume
+
+def test_checkpoint_and_resume_is_bit_exact(mb):
+    """The optimizer's whole state is the weights and the momentum buffers: saving them
+    after two steps and resuming on a fresh handle gives the third step's bits."""
+    import synth
+    data = synth.make_matrix_set(1, layers=[0])
+    G = [g.cuda() for g in data["G"]]
+    W = [w.cuda().clone() for w in data["W"]]
+    M = [m.cuda().clone() for m in data["M"]]
+    h1 = mb.muon_init(0)
+    try:
+        for _ in range(2):
+            mb.muon_step(h1, W, G, M, lr=0.02)
+        torch.cuda.synchronize()
+        saved = {"W": [w.cpu().clone() for w in W], "M": [m.cpu().clone() for m in M]}
+        mb.muon_step(h1, W, G, M, lr=0.02)
+        torch.cuda.synchronize()
+        mb.muon_sync(h1)
+    finally:
+        mb.muon_destroy(h1)
+    W2 = [w.cuda() for w in saved["W"]]
+    M2 = [m.cuda() for m in saved["M"]]
+    h2 = mb.muon_init(0)
+    try:
+        mb.muon_step(h2, W2, G, M2, lr=0.02)
+        torch.cuda.synchronize()
+        mb.muon_sync(h2)
+    finally:
+        mb.muon_destroy(h2)
+    for a, b in zip(W, W2):
+        assert torch.equal(a, b)
+    for a, b in zip(M, M2):
+        assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------- MUON_LOG
+
+def test_log_environment_variable_reports_plans_and_errors():
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import torch, muon_newton_schulz_06_b200 as mb\n"
+        "h = mb.muon_init(0)\n"
+        "w = torch.zeros(300, 100, device='cuda'); g = torch.randn(300, 100, device='cuda')\n"
+        "m = torch.zeros(300, 100, device='cuda')\n"
+        "mb.muon_step(h, [w], [g], [m], lr=0.1); torch.cuda.synchronize()\n"
+        "try:\n"
+        "    mb.muon_step(h, [w], [g], [m], lr=float('nan'))\n"
+        "except mb.MuonError:\n"
+        "    pass\n"
+        "mb.muon_destroy(h)\n")
+    env = dict(os.environ, MUON_LOG="1", PYTHONPATH=root)
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert "muon: plan: 1 matrices" in r.stderr
+    assert "group s=100 L=300 n=1" in r.stderr
+    assert "MUON_ERR_INVALID_ARG" in r.stderr and "lr must be finite" in r.stderr
+    env["MUON_LOG"] = "0"
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and "muon:" not in r.stderr

@@ -72,6 +72,7 @@ def test_reference_arm_runs_on_rank_zero_only():
 # ---------------------------------------------------------------- matrix-sharded step (host logic)
 
 from muon_newton_schulz_06_b200 import sharded  # noqa: E402
+import oracle  # noqa: E402
 import synth  # noqa: E402
 
 
@@ -103,11 +104,24 @@ def test_end_to_end_chunks_cover_the_set_in_balanced_contiguous_runs():
     assert contiguous_chunks([], 4) == []
 
 
-def _fake_step(params, grads, moms, lr=0.1, **kw):
-    # stands in for the CUDA step on CPU: any deterministic in-place update will do
+def _oracle_step(params, grads, moms, lr=0.02, momentum=0.95, **kw):
+    """Stands in for the CUDA step on CPU: the float64 oracle's whole Muon step on each
+    owned matrix (momentum in float32, weights rounded to their dtype)."""
     for w, g, m in zip(params, grads, moms):
-        m.mul_(0.5).add_(g.float())
-        w.sub_(lr * m.to(w.dtype))
+        w_new, m_new, _ = oracle.muon_step_matrix(w.double().numpy(), g.float().numpy(), m.numpy(), lr=lr,
+                                                  mu=momentum, nesterov=True, eps=1e-7)
+        w.copy_(torch.from_numpy(w_new).to(w.dtype))
+        m.copy_(torch.from_numpy(m_new))
+
+
+SHARD_SHAPES = [(6, 4), (4, 6), (8, 8), (10, 3), (3, 10), (5, 5), (12, 12), (16, 9)]
+
+
+def _sharded_inputs():
+    gen = torch.Generator().manual_seed(0)
+    params = [0.02 * torch.randn(r, c, generator=gen) for r, c in SHARD_SHAPES]   # same on every rank
+    grads = [torch.randn(r, c, generator=gen) for r, c in SHARD_SHAPES]
+    return params, grads
 
 
 def _sharded_worker(rank, world, port, out):
@@ -115,32 +129,35 @@ def _sharded_worker(rank, world, port, out):
     import datetime
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=30))
     try:
-        shapes = [(6, 4), (4, 6), (8, 8), (10, 3), (3, 10), (5, 5), (12, 12)]
-        gen = torch.Generator().manual_seed(0)
-        params = [torch.randn(r, c, generator=gen) for r, c in shapes]      # same on every rank
-        grads = [torch.randn(r, c, generator=gen) for r, c in shapes]
-        sm = sharded.ShardedMuon(params, device="cpu", step_fn=_fake_step)
+        params, grads = _sharded_inputs()
+        sm = sharded.ShardedMuon(params, device="cpu", step_fn=_oracle_step)
         for _ in range(3):
-            sm.step([g if sm.owner[i] == rank else None for i, g in enumerate(grads)], lr=0.1)
-        out[rank] = ([p.clone() for p in sm.params], sm.owner, sorted(sm.moms))
+            sm.step([g if sm.owner[i] == rank else None for i, g in enumerate(grads)], lr=0.02, momentum=0.95)
+        out[rank] = ([p.clone() for p in sm.params], sm.owner, sorted(sm.moms),
+                     {i: m.clone() for i, m in sm.moms.items()})
     finally:
         dist.destroy_process_group()
 
 
-def test_sharded_step_gives_every_rank_the_same_updated_weights():
+def test_sharded_step_gives_every_rank_the_oracles_updated_weights():
+    """Two gloo ranks split the matrices by LPT, each runs the oracle's Muon step on its
+    own share, and one all-gather gives both ranks every updated weight: the result
+    equals the oracle's step on every matrix in one process, bit for bit, and momentum
+    lives only on the owning rank."""
     world = 2
     out = mp.Manager().dict()
     mp.spawn(_sharded_worker, args=(world, _free_port(), out), nprocs=world, join=True)
-    # reference: the same fake step on every matrix in one process
-    shapes = [(6, 4), (4, 6), (8, 8), (10, 3), (3, 10), (5, 5), (12, 12)]
-    gen = torch.Generator().manual_seed(0)
-    params = [torch.randn(r, c, generator=gen) for r, c in shapes]
-    grads = [torch.randn(r, c, generator=gen) for r, c in shapes]
-    moms = [torch.zeros(r, c) for r, c in shapes]
+    params, grads = _sharded_inputs()
+    moms = [torch.zeros(r, c) for r, c in SHARD_SHAPES]
     for _ in range(3):
-        _fake_step(params, grads, moms, lr=0.1)
+        _oracle_step(params, grads, moms, lr=0.02, momentum=0.95)
+    owners = set()
     for r in range(world):
-        got, owner, mine = out[r]
+        got, owner, mine, mom = out[r]
         for a, b in zip(got, params):
             assert torch.equal(a, b)
-        assert mine == [i for i in range(len(shapes)) if owner[i] == r]  # momentum only where owned
+        assert mine == [i for i in range(len(SHARD_SHAPES)) if owner[i] == r]  # momentum only where owned
+        for i, m in mom.items():
+            assert torch.equal(m, moms[i])
+        owners |= set(mine)
+    assert owners == set(range(len(SHARD_SHAPES))) and len(set(out[0][1])) == 2
