@@ -71,6 +71,9 @@ def parse():
     ap.add_argument("--cautious", action="store_true", help="decay only where update and weight agree in sign")
     ap.add_argument("--normuon", action="store_true",
                     help="NorMuon rescaling of the orthogonalised update (muon_step_ex, beta2 0.95)")
+    ap.add_argument("--launch-mode", default="auto", choices=["auto", "phases", "persistent"],
+                    help="Newton-Schulz launch form: one launch per phase and step, one persistent launch "
+                         "for all steps, or the library's choice by problem size")
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     return ap.parse_args()
 
@@ -282,6 +285,7 @@ def main():
     torch.cuda.synchronize()
 
     h = mb.muon_init(local)
+    mb.muon_set_launch_mode(h, args.launch_mode)
     stream = torch.cuda.current_stream(dev)
     options, nstate = False, None
     if args.shard:
@@ -385,6 +389,8 @@ def main():
         n_chunks = 1 if args.shard else max(1, min(args.e2e_chunks, len(W)))
         bounds = cost.contiguous_chunks(shapes, n_chunks, NS_STEPS)
         hc = [h] if n_chunks == 1 else [mb.muon_init(local) for _ in bounds]
+        for x in hc:
+            mb.muon_set_launch_mode(x, args.launch_mode)
         g_host = [g.cpu().pin_memory() for g in G]
         w_host = [torch.empty(w.shape, dtype=w.dtype, pin_memory=True) for w in W]
         g_dev = [G, [torch.empty_like(g) for g in G]]
@@ -476,8 +482,9 @@ def main():
         if n == 0:
             continue
         avg_ms = kms / n
-        if kind in ("gram", "poly", "update", "update_apply"):
-            work = fl["per_launch"]["update" if kind == "update_apply" else kind]
+        if kind in ("gram", "poly", "update", "update_apply", "ns_persistent"):
+            work = (fl["algorithmic"] if kind == "ns_persistent"
+                    else fl["per_launch"]["update" if kind == "update_apply" else kind])
             ach = work / (avg_ms / 1e3) / 1e12
             kernels[kind] = {"bound": "tensor", "ms_per_launch": avg_ms, "launches": n, "achieved": ach,
                              "unit": "TFLOP/s", "work_per_launch": work,
@@ -498,7 +505,7 @@ def main():
                 "unit": dk["unit"], "frac": dk["frac"], "traffic": dk["traffic"],
                 "traffic_note": "DRAM bytes per launch (ncu, first layer x 28 layers); null if the kernels "
                                 "changed since the capture"}
-    ns_ms = sum(prof[k][0] for k in ("gram", "poly", "update", "update_apply")) / args.steps
+    ns_ms = sum(prof[k][0] for k in ("gram", "poly", "update", "update_apply", "ns_persistent")) / args.steps
     ns_tflops = fl["algorithmic"] / (ns_ms / 1e3) / 1e12 if ns_ms > 0 else None
 
     # ---------------- CPU oracle on a bounded sample (rank 0, one GPU only)
@@ -522,7 +529,7 @@ def main():
                        **({"options": {"momentum_form": "lerp" if args.lerp else "sgd",
                                        "weight_decay": args.weight_decay, "cautious": args.cautious,
                                        "normuon": args.normuon}} if options else {}),
-                       "nesterov": True, "eps": EPS,
+                       "nesterov": True, "eps": EPS, "launch_mode": args.launch_mode,
                        "l2": "no flush: inputs larger than L2 (%.1f GB of gradients per step)" % (
                            sum(g.numel() * g.element_size() for g in G) / 1e9),
                        "parallelism": ("matrix-sharded, all-gather of new weights" if args.shard else

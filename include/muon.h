@@ -224,6 +224,43 @@ MUON_API muon_status muon_sync(muon_handle_t h);
  * MUON_ERR_INVALID_ARG for a NULL handle or a limit out of range. */
 MUON_API muon_status muon_selftest_wait_timeout(muon_handle_t h, int64_t limit_ns, void* cuda_stream);
 
+/* How the Newton-Schulz steps of a bf16-mode call are launched.  Both forms compute
+ * every tile with the same products in the same order and the same epilogue
+ * arithmetic, so they give the same bits.
+ *  MUON_LAUNCH_PER_PHASE   one grouped launch per phase and step (Gram, polynomial,
+ *                          update; 3 * ns_steps launches per call)
+ *  MUON_LAUNCH_PERSISTENT  one persistent launch for all steps: clusters take work
+ *                          items in order from a global counter, and each item waits
+ *                          (bounded) until its matrix has finished the previous phase, so
+ *                          matrices move through the steps independently and no launch
+ *                          boundary separates the phases.  Used when the call's
+ *                          matrices fall into at most 8 shape groups (otherwise the
+ *                          per-phase form runs)
+ *  MUON_LAUNCH_AUTO        (default) the persistent launch when one Newton-Schulz step
+ *                          over the call's matrices is less than 1e11 algorithmic flops
+ *                          (the smallest sets, where launch boundaries and phase tails
+ *                          weigh most), the per-phase launches otherwise */
+typedef enum {
+  MUON_LAUNCH_AUTO = 0,
+  MUON_LAUNCH_PER_PHASE = 1,
+  MUON_LAUNCH_PERSISTENT = 2
+} muon_launch_mode;
+
+/* Sets the handle's launch form for later calls (no device work).  Returns
+ * MUON_ERR_INVALID_ARG for a NULL handle or an unknown mode. */
+MUON_API muon_status muon_set_launch_mode(muon_handle_t h, muon_launch_mode mode);
+
+/* Diagnostic for the abort path of the persistent launch: in the handle's next
+ * persistent launch, the first polynomial item of the call's first matrix (in the
+ * library's group order) waits for a count that is never reached, with a limit of
+ * limit_ns nanoseconds (1 .. 10e9).  When it runs out, the kernel records a time-out in
+ * the handle's device status; every other item that waits sees the status and gives up,
+ * and the launch returns with its copies and tensor-core work drained.  muon_sync or
+ * the next call then returns MUON_ERR_TIMEOUT (and clears it); the handle keeps
+ * working.  No device work by itself.  Returns MUON_ERR_INVALID_ARG for a NULL handle
+ * or a limit out of range. */
+MUON_API muon_status muon_selftest_stall_persistent(muon_handle_t h, int64_t limit_ns);
+
 /* Diagnostic for the allocation-failure path: the next time the handle must allocate
  * its workspace (a call with a new list of shapes or mode that needs more than the
  * handle holds), the allocation reports failure as if cudaMalloc had failed, once.
@@ -246,7 +283,8 @@ typedef enum {
   MUON_KIND_UPDATE = 3,         /* X' = a X + B X */
   MUON_KIND_APPLY = 4,          /* separate W -= lr*scale*O pass, or the export of O */
   MUON_KIND_UPDATE_APPLY = 5,   /* last update with W -= lr*scale*O fused into its epilogue */
-  MUON_KIND_COUNT = 6
+  MUON_KIND_NS_PERSISTENT = 6,  /* every Newton-Schulz step in one persistent launch */
+  MUON_KIND_COUNT = 7
 } muon_kernel_kind;
 
 /* Per-launch timing: while enabled, every launch of the handle is bracketed by two

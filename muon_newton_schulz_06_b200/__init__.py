@@ -34,12 +34,17 @@ MUON_MODE_FP32_VALIDATE = 1
 
 EXPORTED = ("muon_init", "muon_step", "muon_step_ex", "muon_newton_schulz", "muon_newton_schulz_noalloc",
             "muon_sync",
-            "muon_selftest_wait_timeout", "muon_selftest_fail_next_alloc", "muon_workspace_bytes",
+            "muon_selftest_wait_timeout", "muon_selftest_fail_next_alloc", "muon_selftest_stall_persistent",
+            "muon_set_launch_mode",
+            "muon_workspace_bytes",
             "muon_last_launch_count", "muon_profile_enable", "muon_profile_read", "muon_destroy",
             "muon_status_string", "muon_last_error")
 
 # muon_kernel_kind
-KERNEL_KINDS = ("momentum_norm", "gram", "poly", "update", "apply", "update_apply")
+KERNEL_KINDS = ("momentum_norm", "gram", "poly", "update", "apply", "update_apply", "ns_persistent")
+
+# muon_launch_mode
+LAUNCH_MODES = {"auto": 0, "phases": 1, "persistent": 2}
 
 
 class MuonError(RuntimeError):
@@ -93,6 +98,10 @@ def load_library(path: str = LIB_PATH):
     lib.muon_newton_schulz_noalloc.restype = i32
     lib.muon_selftest_wait_timeout.argtypes = [vp, i64, vp]
     lib.muon_selftest_wait_timeout.restype = i32
+    lib.muon_selftest_stall_persistent.argtypes = [vp, i64]
+    lib.muon_selftest_stall_persistent.restype = i32
+    lib.muon_set_launch_mode.argtypes = [vp, i32]
+    lib.muon_set_launch_mode.restype = i32
     lib.muon_selftest_fail_next_alloc.argtypes = [vp]
     lib.muon_selftest_fail_next_alloc.restype = i32
     lib.muon_sync.argtypes = [vp]
@@ -294,6 +303,21 @@ def muon_selftest_wait_timeout(handle, limit_ns: int, stream=None) -> None:
     """Enqueues the bounded-wait diagnostic (see include/muon.h); the next muon_sync
     raises MuonError with code MUON_ERR_TIMEOUT."""
     _check(load_library().muon_selftest_wait_timeout(handle, int(limit_ns), _stream_ptr(stream, None)), handle)
+
+
+def muon_set_launch_mode(handle, mode: str = "auto") -> None:
+    """How later bf16-mode calls launch the Newton-Schulz steps: "phases" (one grouped
+    launch per phase and step), "persistent" (one launch for all steps) or "auto"."""
+    if mode not in LAUNCH_MODES:
+        raise ValueError(f"unknown launch mode {mode!r}; use one of {sorted(LAUNCH_MODES)}")
+    _check(load_library().muon_set_launch_mode(handle, LAUNCH_MODES[mode]), handle)
+
+
+def muon_selftest_stall_persistent(handle, limit_ns: int) -> None:
+    """Arms the abort-path diagnostic of the persistent launch (see include/muon.h): the
+    handle's next persistent launch gives up after limit_ns and the next muon_sync raises
+    MuonError with code MUON_ERR_TIMEOUT."""
+    _check(load_library().muon_selftest_stall_persistent(handle, int(limit_ns)), handle)
 
 
 def muon_selftest_fail_next_alloc(handle) -> None:

@@ -34,6 +34,7 @@
 // of tile t+1.  Every mbarrier wait is bounded in time; on expiry the kernel writes
 // kDevTimeout to the status word, tells the peer CTA, lets its own copies and MMAs
 // drain, frees TMEM and returns.
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -744,6 +745,529 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
   }
 }
 
+// ---------------------------------------------------------------------- persistent kernel
+//
+// The whole Newton-Schulz loop of one chunk of shape groups in one launch (see
+// TcPersistParams).  Roles as in tc_kernel; what changes:
+//   - work items come from a global counter: the leader's producer takes the next item
+//     (atomicAdd), writes it into an 8-slot ring in both CTAs' shared memory and
+//     arrives on the slot's "full" barrier in both CTAs; every consumer (the peer's
+//     producer, the MMA issuer, the eight epilogue warps) reads the slot and arrives on
+//     the leader's "empty" barrier.  Items are handed out in order, so the lowest
+//     unfinished item always belongs to a running cluster and has no unfinished
+//     dependency: the launch makes progress whatever number of clusters is resident.
+//   - before loading an item's operands, each producer waits (acquire, bounded) until
+//     the item's matrix has finished the previous phase; the epilogue's lane 0 does
+//     the same before its input-block loads.  After its TMA stores of a tile have
+//     completed, each epilogue warp adds 1 (release) to the matrix's counter.
+//   - the phase is a run-time property of the item: operands, descriptors, epilogue
+//     arithmetic and output maps are chosen per item; 4 stages for every phase.
+//   - the epilogue requests all input blocks of its part of a tile (X for Update, A for
+//     Poly; up to 8 blocks of 32 x 32) as soon as it takes the item, and publishes the
+//     previous tile's completion only after that, so one memory latency per tile is
+//     exposed instead of one per chunk.  When the item's inputs are not ready yet, the
+//     previous tile's completion is published first and the wait follows, so no warp
+//     ever waits with an unpublished tile.
+// Every wait is bounded; on expiry, or when another CTA has already recorded a
+// time-out in the status word, the kernel records kDevTimeout, lets its own copies
+// and MMAs drain, frees TMEM and returns.
+constexpr int kPStages = 4;
+constexpr int kSched = 8;  // slots of the work-item ring
+constexpr int kPChunks = kTile / 32 * 4 / kEpiWarps;     // 32-column chunks per epilogue warp and tile
+constexpr uint32_t kPOutPart = 2u * 2u * kOutBlockBytes;  // double-buffered block + mirror
+constexpr uint32_t kPInPart = kPChunks * kOutBlockBytes;  // every input block of the warp's tile part
+constexpr uint32_t kPWarpStage = kPOutPart + kPInPart;
+constexpr uint32_t kPBarrierBytes = 512;
+constexpr uint32_t kPSmemBytes = kPStages * kStageBytes + kEpiWarps * kPWarpStage + kPBarrierBytes + 1024;
+static_assert(kPSmemBytes <= 232448, "shared memory per CTA (persistent kernel)");
+constexpr unsigned kArrivalsPerTile = 2 * kEpiWarps;
+// ring consumers arriving on the leader's empty barrier: the leader's MMA issuer and
+// epilogue warps, the peer's producer and epilogue warps
+constexpr uint32_t kSchedConsumers = 1 + kEpiWarps + 1 + kEpiWarps;
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Orders this thread's generic-proxy global accesses with its async-proxy (TMA) ones.
+__device__ __forceinline__ void fence_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait with cluster-scope acquire (barriers that the other CTA arrives on and
+// whose arrival publishes shared-memory data).
+__device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  uint32_t n = 0;
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((++n & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer() - t0 > kWaitLimitNs) return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void mbar_arrive_local(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// Counter value at which the item's matrix has finished every earlier phase.
+__device__ __forceinline__ unsigned dep_target(const TcGroup& g, int k, int ph) {
+  const int nb = (g.s + kTile - 1) / kTile, nbl = (g.L + kTile - 1) / kTile;
+  const unsigned n_s = (unsigned)(nb * (nb + 1) / 2), n_u = (unsigned)(nb * nbl);
+  const unsigned before = (unsigned)k * (2u * n_s + n_u) + (ph >= kPhasePoly ? n_s : 0u) +
+                          (ph >= kPhaseUpdate ? n_s : 0u);
+  return kArrivalsPerTile * before;
+}
+
+// Waits until *ctr >= target (acquire at GPU scope), bounded; false on time-out, on
+// this CTA's abort flag, or when the status word already records a failure.
+__device__ __noinline__ bool wait_count(const unsigned* ctr, unsigned target, const int* status,
+                                        volatile int* abort_flag, unsigned long long limit_ns = kWaitLimitNs) {
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const uint64_t t0 = global_timer();
+  uint32_t n = 0;
+  while (true) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    if ((++n & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (*reinterpret_cast<const volatile int*>(status) != kDevOk) return false;
+      if (global_timer() - t0 > limit_ns) return false;
+    }
+  }
+}
+
+// Dependency of one item: its matrix's counter must reach the returned value (see
+// TcPersistParams::stall_ns for the self-test form, whose count is never reached).
+__device__ __forceinline__ unsigned item_target(const TcPersistParams& p, const TcGroup& g, int gid, int k, int ph) {
+  if (p.stall_ns != 0 && gid == 0 && k == 0 && ph == kPhasePoly) return 0xffffffffu;
+  return dep_target(g, k, ph);
+}
+__device__ __forceinline__ bool item_ready(const TcPersistParams& p, const TcGroup& g, int gid, int k, int ph) {
+  return ld_acquire_gpu(p.done + gid) >= item_target(p, g, gid, k, ph);
+}
+__device__ __forceinline__ bool wait_item_deps(const TcPersistParams& p, const TcGroup& g, int gid, int k, int ph,
+                                               volatile int* abort_flag) {
+  const unsigned target = item_target(p, g, gid, k, ph);
+  const bool stall = p.stall_ns != 0 && target == 0xffffffffu;
+  return wait_count(p.done + gid, target, p.status, abort_flag, stall ? p.stall_ns : kWaitLimitNs);
+}
+
+// One work item: step k, phase, tile.
+struct PItem {
+  int k, ph;
+  TcTile tile;
+};
+
+__device__ __forceinline__ PItem decode_item(const TcPersistParams& p, int item) {
+  const int per_iter = 2 * p.n_syrk + p.n_upd;
+  PItem it;
+  it.k = item / per_iter;
+  int r = item - it.k * per_iter;
+  if (r < p.n_syrk) {
+    it.ph = kPhaseGram;
+    it.tile = p.tiles_syrk[r];
+  } else if (r < 2 * p.n_syrk) {
+    it.ph = kPhasePoly;
+    it.tile = p.tiles_syrk[r - p.n_syrk];
+  } else {
+    it.ph = kPhaseUpdate;
+    it.tile = p.tiles_upd[r - 2 * p.n_syrk];
+  }
+  return it;
+}
+
+template <typename AppT>
+__global__ void __launch_bounds__(kThreadsTc, 1)
+tc_persistent_kernel(const __grid_constant__ TcPersistParams p, const __grid_constant__ AppT app) {
+  constexpr bool kFuse = sizeof(AppT) > sizeof(TcNoApply);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* out_stage = smem + kPStages * kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPStages * kStageBytes + kEpiWarps * kPWarpStage);
+  uint64_t* empty = full + kPStages;
+  uint64_t* tfull = empty + kPStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint64_t* in_bar = drain + 1;               // [kEpiWarps] input-block barriers
+  uint64_t* sched_full = in_bar + kEpiWarps;
+  uint64_t* sched_empty = sched_full + kSched;  // used in the leader CTA only
+  int* sched_item = reinterpret_cast<int*>(sched_empty + kSched);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sched_item + kSched);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int n_items = p.ns_steps * (2 * p.n_syrk + p.n_upd);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    for (int b = 0; b < kEpiWarps; ++b) mbar_init(&in_bar[b], 1);
+    for (int q = 0; q < kSched; ++q) {
+      mbar_init(&sched_full[q], 1);
+      mbar_init(&sched_empty[q], kSchedConsumers);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t peer_abort = peer_addr(smem_u32((const void*)abort_flag), rank ^ 1u);
+  // the leader's empty barriers, as seen from this CTA (consumers arrive there)
+  const uint32_t leader_sched_empty = peer_addr(smem_u32(&sched_empty[0]), 0);
+
+  auto give_up = [&]() {
+    atomicExch(p.status, kDevTimeout);
+    *abort_flag = 1;
+    remote_store_flag(peer_abort, 1);
+  };
+  // Ring consumer: waits for slot j's item, reads it and releases the slot.
+  auto take_item = [&](uint32_t j, int& item, bool arrive) -> bool {
+    const uint32_t slot = j % kSched, par = (j / kSched) & 1u;
+    if (!mbar_wait_cluster(&sched_full[slot], par, abort_flag)) return false;
+    item = *reinterpret_cast<volatile int*>(&sched_item[slot]);
+    if (arrive) remote_arrive(leader_sched_empty + slot * (uint32_t)sizeof(uint64_t));
+    return true;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (uint32_t j = 0; ok; ++j) {
+        int item;
+        if (rank == 0) {
+          const uint32_t slot = j % kSched, par = (j / kSched) & 1u;
+          if (!mbar_wait_cluster(&sched_empty[slot], par ^ 1u, abort_flag)) { ok = false; break; }
+          item = (int)atomicAdd(p.queue, 1u);
+          if (item >= n_items) item = -1;
+          sched_item[slot] = item;
+          st_cluster_u32(peer_addr(smem_u32(&sched_item[slot]), 1), (uint32_t)item);
+          mbar_arrive_local(&sched_full[slot]);
+          remote_arrive(peer_addr(smem_u32(&sched_full[slot]), 1));
+        } else {
+          if (!take_item(j, item, true)) { ok = false; break; }
+        }
+        if (item < 0) break;
+        const PItem it = decode_item(p, item);
+        const TcGroup& g = p.g[it.tile.group];
+        if (!wait_item_deps(p, g, g.gid_base + it.tile.mat, it.k, it.ph, abort_flag)) { ok = false; break; }
+        fence_async_global();
+        const bool syrk = it.ph != kPhaseUpdate;
+        const int K = (it.ph == kPhaseGram) ? g.L : g.s;
+        const int nk = (K + kBK - 1) / kBK;
+        const int par_x = it.k & 1;
+        const CUtensorMap* ma = it.ph == kPhaseGram ? &p.xk[it.tile.group][par_x]
+                                : it.ph == kPhasePoly ? &p.gram[it.tile.group] : &p.poly[it.tile.group];
+        const CUtensorMap* mb = &p.xmn[it.tile.group][par_x];
+        const int row_a = it.tile.bi * kTile + (int)rank * kHalf;
+        const int col_b = it.tile.bj * kTile + (int)rank * kHalf;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], kPairTxBytes);
+          const uint32_t a_dst = smem_u32(smem + stage * kStageBytes);
+          const uint32_t b_dst = a_dst + kABytes;
+          const uint32_t bar = peer_addr(smem_u32(&full[stage]), 0);
+          const int k0 = kb * kBK;
+          tma_load_3d_pair(a_dst, ma, bar, k0, row_a, it.tile.mat);
+          if (syrk) {
+            tma_load_3d_pair(b_dst, ma, bar, k0, col_b, it.tile.mat);
+          } else {
+#pragma unroll
+            for (int q = 0; q < kHalf / 64; ++q)
+              tma_load_3d_pair(b_dst + q * (64 * kBK * 2), mb, bar, col_b + 64 * q, k0, it.tile.mat);
+          }
+          if (++stage == kPStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok || *abort_flag) {
+        give_up();
+        spin_ns(kAbortGraceNs);  // copies already issued land within microseconds
+      } else if (rank == 0) {
+        for (int s = 0; s < kPStages; ++s) {
+          const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
+          (void)mbar_wait(&full[s], par, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer (leader CTA)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc_k = make_idesc(false), idesc_mn = make_idesc(true);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (uint32_t j = 0; ok; ++j) {
+        int item;
+        if (!take_item(j, item, true)) { ok = false; break; }
+        if (item < 0) break;
+        const PItem it = decode_item(p, item);
+        const TcGroup& g = p.g[it.tile.group];
+        const bool syrk = it.ph != kPhaseUpdate;
+        const int K = (it.ph == kPhaseGram) ? g.L : g.s;
+        const int nk = (K + kBK - 1) / kBK;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kTile);
+        const uint32_t idesc = syrk ? idesc_k : idesc_mn;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
+          const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t ad = sdesc(a_addr + k * 32, 16, 1024);
+            const uint64_t bd = syrk ? sdesc(b_addr + k * 32, 16, 1024) : sdesc(b_addr + k * 2048, 64 * kBK * 2, 1024);
+            umma_pair_bf16(d_tmem, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit_both(&empty[stage]);
+          if (++stage == kPStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_both(&tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) give_up();
+      umma_commit_local(drain);
+      (void)mbar_wait(drain, 0, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (both CTAs)
+    const int quad = warp & 3;
+    const int ew = warp - 2;
+    uint8_t* my_out = out_stage + ew * kPWarpStage;
+    uint8_t* my_in = my_out + kPOutPart;   // kPChunks input blocks
+    uint64_t* my_bar = in_bar + ew;
+    const int c_begin = (ew / 4) * kPChunks;
+    const uint32_t leader_tempty0 = peer_addr(smem_u32(&tempty[0]), 0);
+    uint32_t in_phase = 0;     // parity of my_bar
+    bool in_pending = false;   // input blocks requested and not yet waited for
+    int pend_gid = -1;         // matrix of this warp's last tile, whose completion is unpublished
+    uint32_t n_out = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    // lane 0: the previous tile's stores have landed -> add 1 to its matrix's counter
+    auto publish = [&]() {
+      if (pend_gid >= 0 && lane == 0) {
+        bulk_wait_all();
+        fence_async_global();
+        red_release_gpu_add(p.done + pend_gid, 1u);
+      }
+      pend_gid = -1;
+    };
+    for (uint32_t j = 0; ok; ++j) {
+      int item = -1;
+      bool got = true;
+      if (lane == 0) got = take_item(j, item, true);
+      got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+      item = __shfl_sync(0xffffffffu, item, 0);
+      if (!got) { ok = false; break; }
+      if (item < 0) break;
+      const PItem it = decode_item(p, item);
+      const TcGroup& g = p.g[it.tile.group];
+      const int grp = it.tile.group;
+      const bool syrk = it.ph != kPhaseUpdate;
+      const bool last_update = it.ph == kPhaseUpdate && it.k == p.ns_steps - 1;
+      const int par_x = it.k & 1;
+      const int gid = g.gid_base + it.tile.mat;
+      const int row0 = it.tile.bi * kTile + (int)rank * kHalf + 32 * quad;
+      const int row = row0 + lane;
+      // valid 32-column chunks of this warp: inside the result and, for Gram/Poly, not
+      // strictly below the diagonal
+      int lo = c_begin, hi = c_begin + kPChunks;
+      if (row0 >= g.s) {
+        hi = lo;
+      } else {
+        const int lim = syrk ? g.s : g.L;
+        while (hi > lo && it.tile.bj * kTile + 32 * (hi - 1) >= lim) --hi;
+        if (syrk)
+          while (lo < hi && it.tile.bj * kTile + 32 * lo + 31 < row0) ++lo;
+      }
+      const bool has_in = it.ph != kPhaseGram && lo < hi;
+      const CUtensorMap* map_in = it.ph == kPhasePoly ? &p.gram_out[grp] : &p.xout[grp][par_x];
+      const CUtensorMap* map_out = it.ph == kPhaseGram ? &p.gram_out[grp]
+                                   : it.ph == kPhasePoly ? &p.poly_out[grp] : &p.xout[grp][par_x ^ 1];
+      auto request_all = [&]() {  // lane 0: every input block of chunks [lo, hi), one barrier
+        fence_async_smem();
+        mbar_arrive_expect_tx(my_bar, (uint32_t)(hi - lo) * kOutBlockBytes);
+        for (int c = lo; c < hi; ++c)
+          tma_load_3d_local(smem_u32(my_in + (c - c_begin) * kOutBlockBytes), map_in, my_bar,
+                            it.tile.bj * kTile + 32 * c, row0, it.tile.mat);
+      };
+      if (has_in) {
+        // inputs already complete: request them before publishing the previous tile, so
+        // the two latencies overlap; otherwise publish first, then wait (bounded)
+        int issued = 0;
+        if (lane == 0 && item_ready(p, g, gid, it.k, it.ph)) {
+          fence_async_global();
+          request_all();
+          issued = 1;
+        }
+        issued = __shfl_sync(0xffffffffu, issued, 0);
+        publish();
+        if (!issued) {
+          int dep = 1;
+          if (lane == 0) {
+            dep = wait_item_deps(p, g, gid, it.k, it.ph, abort_flag) ? 1 : 0;
+            if (dep) {
+              fence_async_global();
+              request_all();
+            }
+          }
+          if (__shfl_sync(0xffffffffu, dep, 0) == 0) { ok = false; break; }
+        }
+        in_pending = true;
+      } else {
+        publish();
+      }
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      if (has_in) {
+        if (!mbar_wait(my_bar, in_phase, abort_flag)) { ok = false; break; }
+        in_phase ^= 1u;
+        in_pending = false;
+      }
+      const float sc = it.k == 0 ? p.scale[gid] : 1.f;
+      const uint32_t tbase = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(acc * kTile);
+      for (int c = lo; c < hi; ++c) {
+        const int col0 = it.tile.bj * kTile + 32 * c;
+        float in_v[32];
+        float v[32];
+        tmem_ld32(tbase + (uint32_t)(32 * c), v);
+        if (it.ph == kPhaseGram) {
+          const float alpha = sc * sc;
+#pragma unroll
+          for (int q = 0; q < 32; ++q) v[q] *= alpha;
+        } else if (it.ph == kPhasePoly) {
+          unstage_row(my_in + (c - c_begin) * kOutBlockBytes, lane, in_v);
+          const float cb = p.cb[it.k], cc = p.cc[it.k];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) v[q] = fmaf(cb, in_v[q], cc * v[q]);
+        } else {
+          unstage_row(my_in + (c - c_begin) * kOutBlockBytes, lane, in_v);
+          const float alpha = p.ca[it.k] * sc;
+#pragma unroll
+          for (int q = 0; q < 32; ++q) v[q] = fmaf(alpha, in_v[q], sc * v[q]);
+        }
+        if (!syrk) {
+          if constexpr (kFuse) {
+            if (last_update) {
+              if (row < g.s) {
+                const TcApplyTable& at = reinterpret_cast<const TcApplyTable&>(app);
+                fused_apply_chunk(at.m[gid - at.base], g.s, g.L, row, col0, v);
+              }
+              continue;
+            }
+          }
+          uint8_t* blk = my_out + (n_out & 1) * 2 * kOutBlockBytes;
+          if (lane == 0) bulk_wait_read_1();
+          __syncwarp();
+          stage_row(blk, lane, v);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(map_out, smem_u32(blk), col0, row0, it.tile.mat);
+            bulk_commit();
+          }
+          ++n_out;
+          continue;
+        }
+        uint8_t* blk = my_out + (n_out & 1) * 2 * kOutBlockBytes;
+        if (lane == 0) bulk_wait_read_1();
+        __syncwarp();
+        const bool upper = col0 >= row0 + 32;
+        if (upper) {
+          stage_row(blk, lane, v);
+          uint8_t* mir = blk + kOutBlockBytes;
+#pragma unroll
+          for (int q = 0; q < 32; ++q)
+            *reinterpret_cast<__nv_bfloat16*>(mir + swz64(q, lane)) = __float2bfloat16_rn(v[q]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            if (q >= lane) {
+              const __nv_bfloat16 bv = __float2bfloat16_rn(v[q]);
+              *reinterpret_cast<__nv_bfloat16*>(blk + swz64(lane, q)) = bv;
+              if (q > lane) *reinterpret_cast<__nv_bfloat16*>(blk + swz64(q, lane)) = bv;
+            }
+          }
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(map_out, smem_u32(blk), col0, row0, it.tile.mat);
+          if (upper) tma_store_3d(map_out, smem_u32(blk + kOutBlockBytes), row0, col0, it.tile.mat);
+          bulk_commit();
+        }
+        ++n_out;
+      }
+      tc_fence_before();
+      __syncwarp();  // every lane has read its input rows before the buffer is refilled
+      if (lane == 0) remote_arrive(leader_tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      // the last Update's outputs are read by no later item
+      pend_gid = last_update ? -1 : gid;
+    }
+    if (ok) publish();
+    if (lane == 0) bulk_wait_all();
+    if (!ok && lane == 0) give_up();
+    if (in_pending) (void)mbar_wait(my_bar, in_phase, nullptr);  // requested blocks land before exit
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
 template <int PHASE, typename AppT>
 cudaError_t set_smem_attr() {
   return cudaFuncSetAttribute(tc_kernel<PHASE, AppT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -753,6 +1277,7 @@ cudaError_t set_smem_attr() {
 struct DeviceInfo {
   std::atomic<bool> ready{false};
   int clusters = 0;
+  int persistent_clusters = 0;
 };
 DeviceInfo g_dev_info[64];
 // Serialises the first set-up of a device between host threads (several handles, or
@@ -772,6 +1297,12 @@ cudaError_t device_setup(int dev) {
   if (e == cudaSuccess) e = set_smem_attr<kPhasePoly, TcNoApply>();
   if (e == cudaSuccess) e = set_smem_attr<kPhaseUpdate, TcNoApply>();
   if (e == cudaSuccess) e = set_smem_attr<kPhaseUpdate, TcApplyTable>();
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(tc_persistent_kernel<TcNoApply>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kPSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(tc_persistent_kernel<TcApplyTable>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kPSmemBytes);
   if (e != cudaSuccess) return e;
   int sms = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -794,6 +1325,14 @@ cudaError_t device_setup(int dev) {
     n = sms / 2;
   }
   d.clusters = n;
+  cfg.dynamicSmemBytes = kPSmemBytes;
+  int np = 0;
+  e = cudaOccupancyMaxActiveClusters(&np, tc_persistent_kernel<TcApplyTable>, &cfg);
+  if (e != cudaSuccess || np <= 0) {
+    cudaGetLastError();
+    np = n;
+  }
+  d.persistent_clusters = np;
   d.ready.store(true, std::memory_order_release);
   return cudaSuccess;
 }
@@ -838,6 +1377,35 @@ cudaError_t launch_tc(int phase, const TcParams& p, int clusters, cudaStream_t s
     case kPhaseUpdate: return launch_phase<kPhaseUpdate>(p, none, clusters, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+int tc_persistent_clusters() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || device_setup(dev) != cudaSuccess) return 1;
+  return std::max(1, g_dev_info[dev].persistent_clusters);
+}
+
+cudaError_t launch_tc_persistent(const TcPersistParams& p, const TcApplyTable* app, int clusters, cudaStream_t st) {
+  if (p.n_syrk + p.n_upd == 0 || p.ns_steps == 0) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = device_setup(dev);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
+  cfg.blockDim = dim3(kThreadsTc, 1, 1);
+  cfg.dynamicSmemBytes = kPSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (app) return cudaLaunchKernelEx(&cfg, tc_persistent_kernel<TcApplyTable>, p, *app);
+  const TcNoApply none{0};
+  return cudaLaunchKernelEx(&cfg, tc_persistent_kernel<TcNoApply>, p, none);
 }
 
 cudaError_t launch_wait_selftest(int* status, unsigned long long limit_ns, cudaStream_t st) {

@@ -31,6 +31,9 @@ constexpr float kDefaultCoeffs[3] = {3.4445f, -4.7750f, 2.0315f};
 constexpr int64_t kMaxDim = int64_t(1) << 24;
 constexpr int kMaxNsSteps = 16;
 constexpr int kMaxMatrices = 65535;
+// MUON_LAUNCH_AUTO takes the persistent launch below this algorithmic work of one
+// Newton-Schulz step over all of a call's matrices.
+constexpr double kPersistentMaxFlops = 1e11;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -70,7 +73,7 @@ struct Plan {
   std::vector<int> mat_of_gid;  // caller index of each global (group-major) index
   std::vector<ChunkPlan> chunks;
   std::vector<TcTile> tiles;  // host copy of every chunk's tile lists
-  size_t off_partials = 0, off_scale = 0, off_tiles = 0, off_rowsq = 0, off_rowf = 0, bytes = 0;
+  size_t off_partials = 0, off_scale = 0, off_tiles = 0, off_rowsq = 0, off_rowf = 0, off_sched = 0, bytes = 0;
   int total_rows = 0;
   int total_units = 0;
   // TMA maps per group (bf16 mode): X K-major (ping/pong), X MN-major (ping/pong), Gram, Poly
@@ -115,6 +118,10 @@ struct muon_handle {
   int64_t prof_launches[MUON_KIND_COUNT] = {};
   // muon_selftest_fail_next_alloc: the next workspace allocation reports failure
   bool fail_next_alloc = false;
+  // muon_set_launch_mode
+  int launch_mode = MUON_LAUNCH_AUTO;
+  unsigned long long stall_ns = 0;  // muon_selftest_stall_persistent (next persistent launch)
+  TcPersistParams* persist = nullptr;  // host staging of the persistent launch's parameters
   // MUON_LOG set (and not "0") at muon_init: plan summaries and errors go to stderr
   bool log = false;
 };
@@ -306,6 +313,8 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
   P.off_scale = off; off = align_up(off + (size_t)n * 4, 256);
   P.off_rowsq = off; off = align_up(off + (size_t)P.total_rows * 4, 256);
   P.off_rowf = off; off = align_up(off + (size_t)P.total_rows * 4, 256);
+  // persistent launch: work counter + one completed-tile counter per matrix
+  P.off_sched = off; off = align_up(off + (size_t)(1 + n) * 4, 256);
   // tile lists (tensor-core path)
   if (mode == MUON_MODE_BF16) {
     for (int g0 = 0; g0 < (int)P.groups.size(); g0 += kMaxGroups) {
@@ -728,11 +737,112 @@ bool can_fuse_apply(const Plan& P) {
   return true;
 }
 
+// Fills the handle's fused weight-update table for the matrices of chunk `ch`.
+void fill_apply_table(muon_handle* h, const ChunkPlan& ch, const std::vector<CallMat>& fuse_cm, int cautious) {
+  const Plan& P = h->plan;
+  TcApplyTable& at = *h->apply_table;
+  at.base = P.groups[ch.g_begin].gid_base;
+  const GroupPlan& last = P.groups[ch.g_end - 1];
+  at.n = last.gid_base + last.n - at.base;
+  for (int j = 0; j < at.n; ++j) {
+    const int i = P.mat_of_gid[at.base + j];
+    const CallMat& c = fuse_cm[i];
+    const MatPlan& m = P.mats[i];
+    TcApply& a = at.m[j];
+    a.w = c.param;
+    a.lrs = c.lrs;
+    a.lrwd = c.lrwd;
+    a.flags = (uint16_t)((c.param_bf16 ? kApplyBf16 : 0) | (m.transposed ? kApplyTransposed : 0) |
+                         (m.cols % 8 == 0 ? kApplyVec : 0) | (cautious ? kApplyCautious : 0));
+    a.pad = 0;
+    a.pad2 = 0;
+  }
+}
+
+// True when the whole Newton-Schulz loop of this plan can run as one persistent launch.
+bool can_persist(const Plan& P) {
+  return P.mode == MUON_MODE_BF16 && P.chunks.size() == 1 && P.groups.size() <= (size_t)kMaxGroupsPersist;
+}
+
+// Launch form for this call: the persistent launch removes the per-phase launches and
+// the idle time between phases, which dominates small sets; large sets keep one launch
+// per phase (six operand stages instead of five).
+bool use_persistent(const muon_handle* h, const Plan& P) {
+  if (!can_persist(P)) return false;
+  if (h->launch_mode == MUON_LAUNCH_PERSISTENT) return true;
+  if (h->launch_mode == MUON_LAUNCH_PER_PHASE) return false;
+  double flops = 0.0;  // algorithmic work of one Newton-Schulz step
+  for (const GroupPlan& g : P.groups)
+    flops += (double)g.n * ((double)g.L * g.s * (g.s + 1) + (double)g.s * g.s * (g.s + 1) + 2.0 * g.L * g.s * g.s);
+  return flops < kPersistentMaxFlops;
+}
+
+// The whole Newton-Schulz loop as one persistent launch (see TcPersistParams).
+muon_status launch_ns_persistent(muon_handle* h, const float* coeffs, int ns_steps,
+                                 const std::vector<CallMat>* fuse_cm, int cautious, cudaStream_t st) {
+  const Plan& P = h->plan;
+  const ChunkPlan& ch = P.chunks[0];
+  if (!h->persist) {
+    h->persist = new (std::nothrow) TcPersistParams();
+    if (!h->persist) return fail(h, MUON_ERR_OOM, "host allocation of the persistent-launch parameters failed");
+  }
+  TcPersistParams& pp = *h->persist;
+  std::memset(&pp, 0, sizeof(pp));
+  for (int gg = ch.g_begin; gg < ch.g_end; ++gg) {
+    const int li = gg - ch.g_begin;
+    const GroupPlan& g = P.groups[gg];
+    TcGroup& t = pp.g[li];
+    t.s = g.s; t.L = g.L; t.ld_x = g.ld_x; t.ld_s = g.ld_s; t.gid_base = g.gid_base;
+    t.x_cur = reinterpret_cast<__nv_bfloat16*>(h->ws + g.off_x[0]);
+    t.x_next = reinterpret_cast<__nv_bfloat16*>(h->ws + g.off_x[1]);
+    t.gram = reinterpret_cast<__nv_bfloat16*>(h->ws + g.off_gram);
+    t.poly = reinterpret_cast<__nv_bfloat16*>(h->ws + g.off_poly);
+    for (int b = 0; b < 2; ++b) {
+      pp.xk[li][b] = P.map_xk[b][gg];
+      pp.xmn[li][b] = P.map_xmn[b][gg];
+      pp.xout[li][b] = P.map_xout[b][gg];
+    }
+    pp.gram[li] = P.map_gram[gg];
+    pp.gram_out[li] = P.map_gram_out[gg];
+    pp.poly[li] = P.map_poly[gg];
+    pp.poly_out[li] = P.map_poly_out[gg];
+  }
+  const TcTile* dev_tiles = reinterpret_cast<const TcTile*>(h->ws + P.off_tiles);
+  pp.tiles_syrk = dev_tiles + ch.off_tiles[kPhaseGram];
+  pp.tiles_upd = dev_tiles + ch.off_tiles[kPhaseUpdate];
+  pp.n_syrk = ch.n_tiles[kPhaseGram];
+  pp.n_upd = ch.n_tiles[kPhaseUpdate];
+  pp.ns_steps = ns_steps;
+  for (int k = 0; k < ns_steps; ++k) {
+    const float* c = coeffs ? coeffs + 3 * k : kDefaultCoeffs;
+    pp.ca[k] = c[0];
+    pp.cb[k] = c[1];
+    pp.cc[k] = c[2];
+  }
+  pp.scale = reinterpret_cast<const float*>(h->ws + P.off_scale);
+  pp.status = h->dev_status;
+  pp.queue = reinterpret_cast<unsigned*>(h->ws + P.off_sched);
+  pp.done = pp.queue + 1;
+  pp.stall_ns = h->stall_ns;
+  h->stall_ns = 0;
+  if (fuse_cm) fill_apply_table(h, ch, *fuse_cm, cautious);
+  const int n_items = ns_steps * (2 * pp.n_syrk + pp.n_upd);
+  const int clusters = std::max(1, std::min(tc_persistent_clusters(), n_items));
+  prof_begin(h, st);
+  cudaError_t e = cudaMemsetAsync(pp.queue, 0, (size_t)(1 + P.mats.size()) * 4, st);
+  if (e == cudaSuccess) e = launch_tc_persistent(pp, fuse_cm ? h->apply_table : nullptr, clusters, st);
+  prof_end(h, MUON_KIND_NS_PERSISTENT, st);
+  if (e != cudaSuccess) return cuda_fail(h, e, "persistent Newton-Schulz launch");
+  h->last_launches += 1;
+  return MUON_OK;
+}
+
 // fuse_cm: caller matrices whose weight update is fused into the last Update pass
 // (nullptr: the last pass stores X_K for a separate apply / export pass).
 muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, const std::vector<CallMat>* fuse_cm,
                       int cautious, cudaStream_t st) {
   const Plan& P = h->plan;
+  if (use_persistent(h, P)) return launch_ns_persistent(h, coeffs, ns_steps, fuse_cm, cautious, st);
   float* scale = reinterpret_cast<float*>(h->ws + P.off_scale);
   if (P.mode == MUON_MODE_FP32_VALIDATE) {
     for (int k = 0; k < ns_steps; ++k) {
@@ -803,25 +913,9 @@ muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, const s
         const int clusters = tc_grid_clusters(tp->n_tiles);
         cudaError_t e = cudaSuccess;
         if (fuse_cm && ph == kPhaseUpdate && k == ns_steps - 1) {
-          TcApplyTable& at = *h->apply_table;
-          at.base = P.groups[ch.g_begin].gid_base;
-          const GroupPlan& last = P.groups[ch.g_end - 1];
-          at.n = last.gid_base + last.n - at.base;
-          for (int j = 0; j < at.n; ++j) {
-            const int i = P.mat_of_gid[at.base + j];
-            const CallMat& c = (*fuse_cm)[i];
-            const MatPlan& m = P.mats[i];
-            TcApply& a = at.m[j];
-            a.w = c.param;
-            a.lrs = c.lrs;
-            a.lrwd = c.lrwd;
-            a.flags = (uint16_t)((c.param_bf16 ? kApplyBf16 : 0) | (m.transposed ? kApplyTransposed : 0) |
-                                 (m.cols % 8 == 0 ? kApplyVec : 0) | (cautious ? kApplyCautious : 0));
-            a.pad = 0;
-            a.pad2 = 0;
-          }
+          fill_apply_table(h, ch, *fuse_cm, cautious);
           prof_begin(h, st);
-          e = launch_tc_update_apply(*tp, at, clusters, st);
+          e = launch_tc_update_apply(*tp, *h->apply_table, clusters, st);
           prof_end(h, MUON_KIND_UPDATE_APPLY, st);
         } else {
           prof_begin(h, st);
@@ -1109,6 +1203,22 @@ muon_status muon_selftest_wait_timeout(muon_handle_t h, int64_t limit_ns, void* 
   return finish_call(h, st);
 }
 
+muon_status muon_set_launch_mode(muon_handle_t h, muon_launch_mode mode) {
+  if (!h) return MUON_ERR_INVALID_ARG;
+  if (mode != MUON_LAUNCH_AUTO && mode != MUON_LAUNCH_PER_PHASE && mode != MUON_LAUNCH_PERSISTENT)
+    return fail(h, MUON_ERR_INVALID_ARG, "unknown launch mode %d", (int)mode);
+  h->launch_mode = mode;
+  return MUON_OK;
+}
+
+muon_status muon_selftest_stall_persistent(muon_handle_t h, int64_t limit_ns) {
+  if (!h) return MUON_ERR_INVALID_ARG;
+  h->err.clear();
+  if (limit_ns <= 0 || limit_ns > 10000000000ll) return fail(h, MUON_ERR_INVALID_ARG, "limit_ns out of range");
+  h->stall_ns = (unsigned long long)limit_ns;
+  return MUON_OK;
+}
+
 muon_status muon_selftest_fail_next_alloc(muon_handle_t h) {
   if (!h) return MUON_ERR_INVALID_ARG;
   h->fail_next_alloc = true;
@@ -1176,6 +1286,7 @@ muon_status muon_destroy(muon_handle_t h) {
     for (cudaEvent_t e : h->ev_free) cudaEventDestroy(e);
   }
   delete h->apply_table;
+  delete h->persist;
   delete h;
   return s;
 }

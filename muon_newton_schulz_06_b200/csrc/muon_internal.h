@@ -189,6 +189,52 @@ struct __align__(16) TcApplyTable {
   TcApply m[kMaxFusedApply];
 };
 
+// Whole Newton-Schulz loop in one persistent launch (tc_persistent_kernel): every
+// (step k, phase, tile) item of one chunk of shape groups, in the order
+//   k = 0: Gram tiles, Poly tiles, Update tiles; k = 1: ...
+// is taken from a global work counter by the pair's leader CTA and broadcast to both
+// CTAs' roles.  An item waits until its matrix has finished the previous phase: every
+// epilogue warp of a pair adds 1 to the matrix's counter once its part of a tile is
+// stored, so phase p of step k of a matrix with nS symmetric and nU update tiles may
+// start once the counter reaches kArrivalsPerTile * (k*(2 nS + nU) + [p >= 1] nS +
+// [p >= 2] nS).  The tile lists and their order are those of the per-phase launches,
+// and each tile's products and epilogue arithmetic are the same, so results are
+// bit-identical to launch_tc's.
+constexpr int kMaxNsStepsDev = 16;
+// Shape groups of one persistent launch (ten tensor maps per group travel with it).
+constexpr int kMaxGroupsPersist = 8;
+struct __align__(64) TcPersistParams {
+  CUtensorMap xk[kMaxGroupsPersist][2];   // X (ping, pong) K-major, box 64 x 128: Gram operands
+  CUtensorMap xmn[kMaxGroupsPersist][2];  // X MN-major, box 64 x 64: Update B operand
+  CUtensorMap xout[kMaxGroupsPersist][2]; // X 32 x 32 blocks: Update output and epilogue input
+  CUtensorMap gram[kMaxGroupsPersist];    // Gram K-major: Poly operands
+  CUtensorMap gram_out[kMaxGroupsPersist];// Gram 32 x 32 blocks: Gram output, Poly epilogue input
+  CUtensorMap poly[kMaxGroupsPersist];    // Poly K-major: Update A operand
+  CUtensorMap poly_out[kMaxGroupsPersist];// Poly 32 x 32 blocks: Poly output
+  TcGroup g[kMaxGroupsPersist];
+  const TcTile* tiles_syrk;        // Gram and Poly tiles (cost-sorted), n_syrk entries
+  const TcTile* tiles_upd;         // Update tiles (cost-sorted), n_upd entries
+  int n_syrk, n_upd;
+  int ns_steps;
+  float ca[kMaxNsStepsDev], cb[kMaxNsStepsDev], cc[kMaxNsStepsDev];
+  const float* scale;              // per-matrix 1/(||U||_F + eps)
+  int* status;                     // device status word
+  unsigned* queue;                 // work counter, zero at launch
+  unsigned* done;                  // per-matrix tile arrivals (indexed by gid), zero at launch
+  // self-test of the abort path: when nonzero, the first polynomial item of matrix 0
+  // waits for a count that is never reached, with this limit instead of the usual one
+  unsigned long long stall_ns;
+};
+static_assert(sizeof(TcPersistParams) + sizeof(TcApplyTable) <= 32764,
+              "persistent-kernel parameters must fit the kernel parameter space");
+
+// Launches the persistent kernel with `clusters` 2-CTA clusters (at most the number that
+// fit at once; more items than clusters are fine).  `app` non-null: the last Update
+// applies the weight update in its epilogue instead of storing X_K.
+cudaError_t launch_tc_persistent(const TcPersistParams& p, const TcApplyTable* app, int clusters, cudaStream_t st);
+// Clusters of the persistent kernel that fit on the current device at once.
+int tc_persistent_clusters();
+
 // Number of 2-CTA clusters to launch for n_tiles tiles on the current device.
 int tc_grid_clusters(int n_tiles);
 // Launches 2 * clusters CTAs (one cluster per tile at a time, persistent).
