@@ -74,6 +74,9 @@ def parse():
     ap.add_argument("--launch-mode", default="auto", choices=["auto", "phases", "persistent"],
                     help="Newton-Schulz launch form: one launch per phase and step, one persistent launch "
                          "for all steps, or the library's choice by problem size")
+    ap.add_argument("--mode", default="bf16", choices=["bf16", "fp32", "fp32_simt"],
+                    help="arithmetic of the Newton-Schulz steps: bf16 tensor cores (the method's mode), fp32 "
+                         "validation on tensor cores (3xTF32), or fp32 validation on CUDA cores")
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     return ap.parse_args()
 
@@ -99,6 +102,7 @@ def measured_traffic(config, layers):
     with open(path) as f:
         t = json.load(f)
     files = sorted(glob.glob(os.path.join(ROOT, "muon_newton_schulz_06_b200", "csrc", "*.cu")) +
+                   glob.glob(os.path.join(ROOT, "muon_newton_schulz_06_b200", "csrc", "*.cuh")) +
                    glob.glob(os.path.join(ROOT, "muon_newton_schulz_06_b200", "csrc", "*.h")))
     h = hashlib.sha256()
     for fn in files:
@@ -295,7 +299,8 @@ def main():
         del M
 
         def step(grads=G, st=None):
-            sm.step(grads, lr=LR, momentum=MU, nesterov=True, ns_steps=NS_STEPS, eps=EPS, stream=st or stream)
+            sm.step(grads, lr=LR, momentum=MU, nesterov=True, ns_steps=NS_STEPS, eps=EPS, mode=args.mode,
+                    stream=st or stream)
     else:
         sm = None
 
@@ -306,10 +311,10 @@ def main():
             if options:
                 mb.muon_step_ex(h, W, grads, M, lr=LR, momentum=MU, nesterov=True, ns_steps=NS_STEPS, eps=EPS,
                                 momentum_form="lerp" if args.lerp else "sgd", weight_decay=args.weight_decay,
-                                cautious=args.cautious, normuon_state=nstate, stream=st or stream)
+                                cautious=args.cautious, normuon_state=nstate, mode=args.mode, stream=st or stream)
             else:
                 mb.muon_step(h, W, grads, M, lr=LR, momentum=MU, nesterov=True, ns_steps=NS_STEPS, eps=EPS,
-                             stream=st or stream)
+                             mode=args.mode, stream=st or stream)
 
     for _ in range(max(args.warmup, 0)):
         step()
@@ -411,10 +416,11 @@ def main():
                 mb.muon_step_ex(hc[c], W[a:b], grads[a:b], M[a:b], lr=LR, momentum=MU, nesterov=True,
                                 ns_steps=NS_STEPS, eps=EPS, momentum_form="lerp" if args.lerp else "sgd",
                                 weight_decay=args.weight_decay, cautious=args.cautious,
-                                normuon_state=nstate[a:b] if nstate is not None else None, stream=st)
+                                normuon_state=nstate[a:b] if nstate is not None else None, mode=args.mode,
+                                stream=st)
             else:
                 mb.muon_step(hc[c], W[a:b], grads[a:b], M[a:b], lr=LR, momentum=MU, nesterov=True,
-                             ns_steps=NS_STEPS, eps=EPS, stream=st)
+                             ns_steps=NS_STEPS, eps=EPS, mode=args.mode, stream=st)
 
         def upload(k, c):
             a, b = bounds[c]
@@ -520,7 +526,8 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-            "scaling": "strong" if args.shard else "weak", "vs_baseline": None, "dtype": "bf16",
+            "scaling": "strong" if args.shard else "weak", "vs_baseline": None,
+            "dtype": "bf16" if args.mode == "bf16" else "f32",
             "data": "synthetic",
             "config": {"workload": WORKLOAD_TEXT[cfg] + (f" (first {args.layers} layers only)" if args.layers
                                                           else ""), "matrices": len(shapes),
@@ -529,7 +536,7 @@ def main():
                        **({"options": {"momentum_form": "lerp" if args.lerp else "sgd",
                                        "weight_decay": args.weight_decay, "cautious": args.cautious,
                                        "normuon": args.normuon}} if options else {}),
-                       "nesterov": True, "eps": EPS, "launch_mode": args.launch_mode,
+                       "nesterov": True, "eps": EPS, "launch_mode": args.launch_mode, "mode": args.mode,
                        "l2": "no flush: inputs larger than L2 (%.1f GB of gradients per step)" % (
                            sum(g.numel() * g.element_size() for g in G) / 1e9),
                        "parallelism": ("matrix-sharded, all-gather of new weights" if args.shard else

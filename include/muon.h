@@ -16,9 +16,10 @@
  * The page fixes the momentum, the five Newton-Schulz steps, the tall/wide rules
  * and per-step coefficient triples ("Polar Express", values not printed); the
  * Frobenius normalisation with eps and the update scale come from the method's
- * task statement.  Newton-Schulz runs on tcgen05 tensor cores (bf16 operands,
- * fp32 accumulation) in MUON_MODE_BF16 and on fp32 CUDA-core FMAs in
- * MUON_MODE_FP32_VALIDATE.
+ * task statement.  Newton-Schulz runs on tcgen05 tensor cores with bf16 operands and
+ * fp32 accumulation in MUON_MODE_BF16, on tcgen05 tensor cores with fp32 storage and
+ * 3xTF32 products in MUON_MODE_FP32_VALIDATE, and on fp32 CUDA-core FMAs in
+ * MUON_MODE_FP32_SIMT.
  *
  * Conventions for every entry point
  *  - All matrix pointers are DEVICE pointers on the handle's device, row-major and
@@ -74,8 +75,11 @@ typedef enum {
 typedef enum { MUON_F32 = 0, MUON_BF16 = 1 } muon_dtype;
 
 typedef enum {
-  MUON_MODE_BF16 = 0,          /* Newton-Schulz on tcgen05 tensor cores, bf16 operands, fp32 accumulate */
-  MUON_MODE_FP32_VALIDATE = 1  /* Newton-Schulz in fp32 storage and fp32 FMA (validation, slow) */
+  MUON_MODE_BF16 = 0,           /* Newton-Schulz on tcgen05 tensor cores, bf16 operands, fp32 accumulate */
+  MUON_MODE_FP32_VALIDATE = 1,  /* fp32 storage; products on tcgen05 tensor cores as 3xTF32: each fp32
+                                   value is split into hi = tf32(x) and lo = tf32(x - hi) and a
+                                   product accumulates hi*hi + hi*lo + lo*hi in fp32 (validation) */
+  MUON_MODE_FP32_SIMT = 2       /* fp32 storage and fp32 FMA on CUDA cores (validation, slowest) */
 } muon_mode;
 
 /* One weight matrix.  param: rows*cols of param_dtype, updated in place.  grad:
@@ -105,7 +109,7 @@ MUON_API muon_status muon_init(muon_handle_t* out, int device);
  *                Newton-Schulz step k; NULL = (3.4445, -4.7750, 2.0315) every step
  *  ns_steps      1..16
  *  eps           added to the Frobenius norm (finite, >= 0)
- *  mode          MUON_MODE_BF16 or MUON_MODE_FP32_VALIDATE
+ *  mode          MUON_MODE_BF16, MUON_MODE_FP32_VALIDATE or MUON_MODE_FP32_SIMT
  *  cuda_stream   cudaStream_t the work is enqueued on
  * Every matrix is processed independently; their order does not matter.  The
  * applied factor per matrix is the float32 rounding of lr*sqrt(max(1,rows/cols))
@@ -237,9 +241,9 @@ MUON_API muon_status muon_selftest_wait_timeout(muon_handle_t h, int64_t limit_n
  *                          matrices fall into at most 8 shape groups (otherwise the
  *                          per-phase form runs)
  *  MUON_LAUNCH_AUTO        (default) the persistent launch when one Newton-Schulz step
- *                          over the call's matrices is less than 1e11 algorithmic flops
- *                          (the smallest sets, where launch boundaries and phase tails
- *                          weigh most), the per-phase launches otherwise */
+ *                          over the call's matrices is less than 1e12 algorithmic flops
+ *                          (the small sets, where launch boundaries and phase tails weigh
+ *                          most), the per-phase launches otherwise */
 typedef enum {
   MUON_LAUNCH_AUTO = 0,
   MUON_LAUNCH_PER_PHASE = 1,

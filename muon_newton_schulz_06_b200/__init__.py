@@ -31,6 +31,7 @@ MUON_F32 = 0
 MUON_BF16 = 1
 MUON_MODE_BF16 = 0
 MUON_MODE_FP32_VALIDATE = 1
+MUON_MODE_FP32_SIMT = 2
 
 EXPORTED = ("muon_init", "muon_step", "muon_step_ex", "muon_newton_schulz", "muon_newton_schulz_noalloc",
             "muon_sync",
@@ -164,6 +165,8 @@ def _mode_code(mode) -> int:
         return MUON_MODE_BF16
     if mode in ("fp32", "fp32_validate", MUON_MODE_FP32_VALIDATE):
         return MUON_MODE_FP32_VALIDATE
+    if mode in ("fp32_simt", MUON_MODE_FP32_SIMT):
+        return MUON_MODE_FP32_SIMT
     raise ValueError(f"unknown mode {mode!r}")
 
 

@@ -39,6 +39,7 @@
 #include <mutex>
 
 #include "muon_internal.h"
+#include "tc_primitives.cuh"
 
 namespace muon {
 namespace {
@@ -65,72 +66,11 @@ __host__ __device__ constexpr uint32_t smem_bytes_for(int phase) {
 }
 static_assert(smem_bytes_for(0) <= 232448 && smem_bytes_for(1) <= 232448 && smem_bytes_for(2) <= 232448,
               "shared memory per CTA");
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
-constexpr unsigned long long kAbortGraceNs = 1000000ull;    // 1 ms for copies in flight
 
 // tcgen05 instruction descriptor, kind::f16: D f32, A/B bf16, A K-major, M = N = 256.
 __host__ __device__ constexpr uint32_t make_idesc(bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
          ((uint32_t)(kTile >> 3) << 17) | ((uint32_t)(kTile >> 4) << 24);
-}
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// Shared-memory matrix descriptor (sm_100 format): start, leading / stride byte
-// offsets (16-byte units), version 1, 128-byte swizzle.
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
-}
-
-__device__ __forceinline__ uint64_t global_timer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait: false after limit_ns, or (when abort_flag is given) once another role of
-// the CTA gave up.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                       unsigned long long limit_ns = kWaitLimitNs) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer();
-  uint32_t n = 0;
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((++n & 63u) == 0) {
-      if (abort_flag != nullptr && *abort_flag) return false;
-      if (global_timer() - t0 > limit_ns) return false;
-    }
-  }
 }
 
 // Diagnostic: one thread waits, with the same bounded wait as the engine, on a barrier
@@ -144,43 +84,6 @@ __global__ void wait_selftest_kernel(int* status, unsigned long long limit_ns) {
   }
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-// Address of the same shared-memory location in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t peer_addr(uint32_t saddr, uint32_t rank) {
-  uint32_t out;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(saddr), "r"(rank));
-  return out;
-}
-
-__device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
-__device__ __forceinline__ void remote_store_flag(uint32_t cluster_addr, int v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Bulk tensor copy into this CTA's shared memory whose completion is counted on the
-// barrier at `bar_cluster_addr` (the leader CTA's).  No multicast.
-__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster_addr,
-                                                 int x, int y, int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-
 __device__ __forceinline__ void umma_pair_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                                uint32_t accumulate) {
   asm volatile(
@@ -188,32 +91,6 @@ __device__ __forceinline__ void umma_pair_bf16(uint32_t d_tmem, uint64_t adesc, 
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
-}
-
-// Arrives on the barrier at the same offset in both CTAs once this thread's MMAs finish.
-__device__ __forceinline__ void umma_commit_both(uint64_t* bar) {
-  const uint16_t mask = 0x3;
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-          smem_u32(bar)),
-      "h"(mask)
-      : "memory");
-}
-
-// Arrives on this CTA's barrier once this thread's MMAs finish.
-__device__ __forceinline__ void umma_commit_local(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-// Bulk tensor copy into this CTA's shared memory, completing on this CTA's barrier.
-__device__ __forceinline__ void tma_load_3d_local(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int x,
-                                                  int y, int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
-      : "memory");
 }
 
 // Thread `r` reads row r of a staged 32 x 32 bf16 block (4 x 16-byte loads).
@@ -231,19 +108,6 @@ __device__ __forceinline__ void unstage_row(const uint8_t* blk, int r, float* v)
   }
 }
 
-// Bulk tensor store of a shared-memory block (tile mode; out-of-range parts are clipped).
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y, int z) {
-  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(src), "r"(x), "r"(y), "r"(z)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// At most one committed store group may still be reading shared memory.
-__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
 // Byte offset of element (r, c) in a 32 x 32 bf16 block with 64-byte rows under the
 // 64-byte swizzle: the 16-byte chunk index is XORed with bits 1..2 of the row.
 __device__ __forceinline__ uint32_t swz64(int r, int c) {
@@ -260,37 +124,6 @@ __device__ __forceinline__ void stage_row(uint8_t* blk, int r, const float* v) {
     for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(v[8 * q + 2 * e], v[8 * q + 2 * e + 1]);
     *reinterpret_cast<uint4*>(blk + r * 64 + (((q ^ (r >> 1)) & 3) << 4)) = raw;
   }
-}
-
-__device__ __forceinline__ void spin_ns(unsigned long long ns) {
-  const uint64_t t0 = global_timer();
-  while (global_timer() - t0 < ns) {
-  }
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// 32 lanes x 32 consecutive fp32 columns: thread i gets row (lane base + i).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float* v) {
@@ -337,10 +170,11 @@ __device__ __forceinline__ float apply_one(float w0, float o, float lrs, float l
 
 template <typename WT>
 __device__ __forceinline__ void fused_apply_chunk_t(WT* w, float lrs, float lrwd, bool cautious, bool transposed,
-                                                    bool vec, int s, int L, int row, int col0, const float* xv) {
-  float o[32], wv[32];
+                                                    bool vec, int s, int L, int row, int col0, float* o) {
+  float wv[32];
+  // O = bf16(X_K), in place
 #pragma unroll
-  for (int j = 0; j < 32; ++j) o[j] = __bfloat162float(__float2bfloat16_rn(xv[j]));
+  for (int j = 0; j < 32; ++j) o[j] = __bfloat162float(__float2bfloat16_rn(o[j]));
   if (!transposed && vec && col0 + 32 <= L) {
     // W is s x L: this thread's 32 consecutive entries of row `row`
     WT* p = w + (size_t)row * L + col0;
@@ -401,8 +235,8 @@ __device__ __forceinline__ void fused_apply_chunk_t(WT* w, float lrs, float lrwd
   }
 }
 
-__device__ __forceinline__ void fused_apply_chunk(const TcApply& ap, int s, int L, int row, int col0,
-                                                  const float* xv) {
+// xv: X_K of the chunk in fp32, overwritten with O = bf16(X_K).
+__device__ __forceinline__ void fused_apply_chunk(const TcApply& ap, int s, int L, int row, int col0, float* xv) {
   const bool tr = ap.flags & kApplyTransposed, vec = ap.flags & kApplyVec, ca = ap.flags & kApplyCautious;
   if (ap.flags & kApplyBf16)
     fused_apply_chunk_t(reinterpret_cast<__nv_bfloat16*>(ap.w), ap.lrs, ap.lrwd, ca, tr, vec, s, L, row, col0, xv);
@@ -762,8 +596,12 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
 //     completed, each epilogue warp adds 1 (release) to the matrix's counter.
 //   - the phase is a run-time property of the item: operands, descriptors, epilogue
 //     arithmetic and output maps are chosen per item; 4 stages for every phase.
+//   - eight epilogue warps, two per TMEM lane quadrant, each with half of the tile's
+//     columns, so two warps per scheduler hide each other's latencies; one output
+//     staging buffer per warp (the other warp on its scheduler covers the wait for the
+//     previous store to leave it).
 //   - the epilogue requests all input blocks of its part of a tile (X for Update, A for
-//     Poly; up to 8 blocks of 32 x 32) as soon as it takes the item, and publishes the
+//     Poly; 4 blocks of 32 x 32) as soon as it takes the item, and publishes the
 //     previous tile's completion only after that, so one memory latency per tile is
 //     exposed instead of one per chunk.  When the item's inputs are not ready yet, the
 //     previous tile's completion is published first and the wait follows, so no warp
@@ -772,18 +610,20 @@ tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ AppT app) 
 // time-out in the status word, the kernel records kDevTimeout, lets its own copies
 // and MMAs drain, frees TMEM and returns.
 constexpr int kPStages = 4;
+constexpr int kPEpi = 8;                                  // epilogue warps: two per TMEM lane quadrant
+constexpr int kPThreads = 64 + 32 * kPEpi;
 constexpr int kSched = 8;  // slots of the work-item ring
-constexpr int kPChunks = kTile / 32 * 4 / kEpiWarps;     // 32-column chunks per epilogue warp and tile
-constexpr uint32_t kPOutPart = 2u * 2u * kOutBlockBytes;  // double-buffered block + mirror
+constexpr int kPChunks = kTile / 32 * 4 / kPEpi;          // 32-column chunks per epilogue warp and tile
+constexpr uint32_t kPOutPart = 2u * kOutBlockBytes;       // one block + its mirror
 constexpr uint32_t kPInPart = kPChunks * kOutBlockBytes;  // every input block of the warp's tile part
 constexpr uint32_t kPWarpStage = kPOutPart + kPInPart;
 constexpr uint32_t kPBarrierBytes = 512;
-constexpr uint32_t kPSmemBytes = kPStages * kStageBytes + kEpiWarps * kPWarpStage + kPBarrierBytes + 1024;
+constexpr uint32_t kPSmemBytes = kPStages * kStageBytes + kPEpi * kPWarpStage + kPBarrierBytes + 1024;
 static_assert(kPSmemBytes <= 232448, "shared memory per CTA (persistent kernel)");
-constexpr unsigned kArrivalsPerTile = 2 * kEpiWarps;
+constexpr unsigned kArrivalsPerTile = 2 * kPEpi;
 // ring consumers arriving on the leader's empty barrier: the leader's MMA issuer and
 // epilogue warps, the peer's producer and epilogue warps
-constexpr uint32_t kSchedConsumers = 1 + kEpiWarps + 1 + kEpiWarps;
+constexpr uint32_t kSchedConsumers = 1 + kPEpi + 1 + kPEpi;
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
@@ -793,6 +633,8 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
 __device__ __forceinline__ void red_release_gpu_add(unsigned* p, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// Every committed store group of this thread has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Orders this thread's generic-proxy global accesses with its async-proxy (TMA) ones.
 __device__ __forceinline__ void fence_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
@@ -899,19 +741,19 @@ __device__ __forceinline__ PItem decode_item(const TcPersistParams& p, int item)
 }
 
 template <typename AppT>
-__global__ void __launch_bounds__(kThreadsTc, 1)
+__global__ void __launch_bounds__(kPThreads, 1)
 tc_persistent_kernel(const __grid_constant__ TcPersistParams p, const __grid_constant__ AppT app) {
   constexpr bool kFuse = sizeof(AppT) > sizeof(TcNoApply);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* out_stage = smem + kPStages * kStageBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPStages * kStageBytes + kEpiWarps * kPWarpStage);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPStages * kStageBytes + kPEpi * kPWarpStage);
   uint64_t* empty = full + kPStages;
   uint64_t* tfull = empty + kPStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint64_t* in_bar = drain + 1;               // [kEpiWarps] input-block barriers
-  uint64_t* sched_full = in_bar + kEpiWarps;
+  uint64_t* in_bar = drain + 1;               // [kPEpi] input-block barriers
+  uint64_t* sched_full = in_bar + kPEpi;
   uint64_t* sched_empty = sched_full + kSched;  // used in the leader CTA only
   int* sched_item = reinterpret_cast<int*>(sched_empty + kSched);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sched_item + kSched);
@@ -929,10 +771,10 @@ tc_persistent_kernel(const __grid_constant__ TcPersistParams p, const __grid_con
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 2 * kEpiWarps);
+      mbar_init(&tempty[a], 2 * kPEpi);
     }
     mbar_init(drain, 1);
-    for (int b = 0; b < kEpiWarps; ++b) mbar_init(&in_bar[b], 1);
+    for (int b = 0; b < kPEpi; ++b) mbar_init(&in_bar[b], 1);
     for (int q = 0; q < kSched; ++q) {
       mbar_init(&sched_full[q], 1);
       mbar_init(&sched_empty[q], kSchedConsumers);
@@ -1086,7 +928,6 @@ tc_persistent_kernel(const __grid_constant__ TcPersistParams p, const __grid_con
     uint32_t in_phase = 0;     // parity of my_bar
     bool in_pending = false;   // input blocks requested and not yet waited for
     int pend_gid = -1;         // matrix of this warp's last tile, whose completion is unpublished
-    uint32_t n_out = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
@@ -1203,8 +1044,8 @@ tc_persistent_kernel(const __grid_constant__ TcPersistParams p, const __grid_con
               continue;
             }
           }
-          uint8_t* blk = my_out + (n_out & 1) * 2 * kOutBlockBytes;
-          if (lane == 0) bulk_wait_read_1();
+          uint8_t* blk = my_out;  // single staging buffer: the previous store has read it
+          if (lane == 0) bulk_wait_read_0();
           __syncwarp();
           stage_row(blk, lane, v);
           fence_async_smem();
@@ -1213,11 +1054,10 @@ tc_persistent_kernel(const __grid_constant__ TcPersistParams p, const __grid_con
             tma_store_3d(map_out, smem_u32(blk), col0, row0, it.tile.mat);
             bulk_commit();
           }
-          ++n_out;
           continue;
         }
-        uint8_t* blk = my_out + (n_out & 1) * 2 * kOutBlockBytes;
-        if (lane == 0) bulk_wait_read_1();
+        uint8_t* blk = my_out;
+        if (lane == 0) bulk_wait_read_0();
         __syncwarp();
         const bool upper = col0 >= row0 + 32;
         if (upper) {
@@ -1243,7 +1083,6 @@ tc_persistent_kernel(const __grid_constant__ TcPersistParams p, const __grid_con
           if (upper) tma_store_3d(map_out, smem_u32(blk + kOutBlockBytes), row0, col0, it.tile.mat);
           bulk_commit();
         }
-        ++n_out;
       }
       tc_fence_before();
       __syncwarp();  // every lane has read its input rows before the buffer is refilled
@@ -1325,6 +1164,7 @@ cudaError_t device_setup(int dev) {
     n = sms / 2;
   }
   d.clusters = n;
+  cfg.blockDim = dim3(kPThreads, 1, 1);
   cfg.dynamicSmemBytes = kPSmemBytes;
   int np = 0;
   e = cudaOccupancyMaxActiveClusters(&np, tc_persistent_kernel<TcApplyTable>, &cfg);
@@ -1393,7 +1233,7 @@ cudaError_t launch_tc_persistent(const TcPersistParams& p, const TcApplyTable* a
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
-  cfg.blockDim = dim3(kThreadsTc, 1, 1);
+  cfg.blockDim = dim3(kPThreads, 1, 1);
   cfg.dynamicSmemBytes = kPSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];

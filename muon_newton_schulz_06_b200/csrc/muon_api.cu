@@ -33,7 +33,7 @@ constexpr int kMaxNsSteps = 16;
 constexpr int kMaxMatrices = 65535;
 // MUON_LAUNCH_AUTO takes the persistent launch below this algorithmic work of one
 // Newton-Schulz step over all of a call's matrices.
-constexpr double kPersistentMaxFlops = 1e11;
+constexpr double kPersistentMaxFlops = 1e12;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -48,6 +48,9 @@ struct GroupPlan {
   int gid_base = 0;
   size_t off_x[2] = {0, 0};
   size_t off_gram = 0, off_poly = 0;
+  // 3xTF32 mode: the lo parts (the arrays above hold the hi parts)
+  size_t off_xlo[2] = {0, 0};
+  size_t off_gram_lo = 0, off_poly_lo = 0;
 };
 
 struct MatPlan {
@@ -80,6 +83,8 @@ struct Plan {
   std::vector<CUtensorMap> map_xk[2], map_xmn[2], map_gram, map_poly;
   // output maps (32 x 32 boxes, 64-byte swizzle) for the epilogue's TMA stores
   std::vector<CUtensorMap> map_xout[2], map_gram_out, map_poly_out;
+  // 3xTF32 mode (fp32): X K-major and MN-major, Gram, Poly; hi and lo parts
+  std::vector<CUtensorMap> t_xk[2][2], t_xmn[2][2], t_gram[2], t_poly[2];
 };
 
 }  // namespace
@@ -224,12 +229,14 @@ void sort_tiles(std::vector<TcTile>& t, const std::vector<GroupPlan>& groups, in
 
 muon_status encode_map(muon_handle* h, CUtensorMap* map, void* base, int inner, int rows, int n, int ld,
                        int box_inner, int box_rows,
-                       CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+                       CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B, bool f32 = false) {
+  const cuuint64_t esz = f32 ? 4 : 2;
   cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)n};
-  cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)ld * 2 * (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * esz, (cuuint64_t)ld * esz * (cuuint64_t)rows};
   cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = h->encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+  CUresult r = h->encode(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base,
+                         dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(h, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -301,6 +308,7 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
   }
   // workspace layout
   size_t off = 0;
+  const bool tf32x3 = mode == MUON_MODE_FP32_VALIDATE;
   for (auto& g : P.groups) {
     const size_t xbytes = (size_t)g.n * g.s * g.ld_x * esz;
     const size_t sbytes = (size_t)g.n * g.s * g.ld_s * esz;
@@ -308,6 +316,12 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
     g.off_x[1] = off; off = align_up(off + xbytes, 1024);
     g.off_gram = off; off = align_up(off + sbytes, 1024);
     g.off_poly = off; off = align_up(off + sbytes, 1024);
+    if (tf32x3) {
+      g.off_xlo[0] = off; off = align_up(off + xbytes, 1024);
+      g.off_xlo[1] = off; off = align_up(off + xbytes, 1024);
+      g.off_gram_lo = off; off = align_up(off + sbytes, 1024);
+      g.off_poly_lo = off; off = align_up(off + sbytes, 1024);
+    }
   }
   P.off_partials = off; off = align_up(off + (size_t)P.total_units * kWarpsPerUnit * 4, 256);
   P.off_scale = off; off = align_up(off + (size_t)n * 4, 256);
@@ -315,8 +329,8 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
   P.off_rowf = off; off = align_up(off + (size_t)P.total_rows * 4, 256);
   // persistent launch: work counter + one completed-tile counter per matrix
   P.off_sched = off; off = align_up(off + (size_t)(1 + n) * 4, 256);
-  // tile lists (tensor-core path)
-  if (mode == MUON_MODE_BF16) {
+  // tile lists (tensor-core paths)
+  if (mode != MUON_MODE_FP32_SIMT) {
     for (int g0 = 0; g0 < (int)P.groups.size(); g0 += kMaxGroups) {
       ChunkPlan c;
       c.g_begin = g0;
@@ -407,6 +421,35 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
         return s;
     }
   }
+  if (tf32x3) {
+    const size_t ng = P.groups.size();
+    for (int part = 0; part < 2; ++part) {
+      for (int b = 0; b < 2; ++b) {
+        P.t_xk[part][b].resize(ng);
+        P.t_xmn[part][b].resize(ng);
+      }
+      P.t_gram[part].resize(ng);
+      P.t_poly[part].resize(ng);
+    }
+    const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    for (size_t gg = 0; gg < ng; ++gg) {
+      const GroupPlan& g = P.groups[gg];
+      muon_status s;
+      for (int part = 0; part < 2; ++part) {
+        for (int b = 0; b < 2; ++b) {
+          char* xb = h->ws + (part == 0 ? g.off_x[b] : g.off_xlo[b]);
+          if ((s = encode_map(h, &P.t_xk[part][b][gg], xb, g.L, g.s, g.n, g.ld_x, 32, kHalf, sw, true))) return s;
+          if ((s = encode_map(h, &P.t_xmn[part][b][gg], xb, g.L, g.s, g.n, g.ld_x, 32, 32,
+                              CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B, true)))
+            return s;
+        }
+        char* gb = h->ws + (part == 0 ? g.off_gram : g.off_gram_lo);
+        char* pb = h->ws + (part == 0 ? g.off_poly : g.off_poly_lo);
+        if ((s = encode_map(h, &P.t_gram[part][gg], gb, g.s, g.s, g.n, g.ld_s, 32, kHalf, sw, true))) return s;
+        if ((s = encode_map(h, &P.t_poly[part][gg], pb, g.s, g.s, g.n, g.ld_s, 32, kHalf, sw, true))) return s;
+      }
+    }
+  }
   P.valid = true;
   if (h->log) {
     size_t n_tiles[3] = {0, 0, 0};
@@ -416,7 +459,7 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
             "muon: plan: %d matrices, %zu shape groups, %zu launch chunks, tiles gram/poly/update %zu/%zu/%zu, "
             "workspace %zu bytes (%s mode)\n",
             n, P.groups.size(), P.chunks.size(), n_tiles[0], n_tiles[1], n_tiles[2], P.bytes,
-            mode == MUON_MODE_BF16 ? "bf16" : "fp32");
+            mode == MUON_MODE_BF16 ? "bf16" : mode == MUON_MODE_FP32_VALIDATE ? "fp32 3xTF32" : "fp32 CUDA-core");
     for (const GroupPlan& g : P.groups) fprintf(stderr, "muon:   group s=%d L=%d n=%d\n", g.s, g.L, g.n);
   }
   return MUON_OK;
@@ -654,7 +697,7 @@ muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, i
   const int nesterov = o.nesterov;
   const Plan& P = h->plan;
   const int n = (int)cm.size();
-  const bool f32 = (P.mode == MUON_MODE_FP32_VALIDATE);
+  const bool f32 = (P.mode != MUON_MODE_BF16);
   for (int b = 0; b < n; b += kMaxMatsPerLaunch) {
     EwParams* ep = new EwParams();
     std::memset(ep, 0, sizeof(EwParams));
@@ -837,6 +880,76 @@ muon_status launch_ns_persistent(muon_handle* h, const float* coeffs, int ns_ste
   return MUON_OK;
 }
 
+// fp32 validation mode on the tensor cores (3xTF32): split X0 into its hi and lo parts,
+// then one grouped launch per phase and step; the last Update stores X_K unsplit for the
+// weight-update / export pass.
+muon_status launch_ns_tf32x3(muon_handle* h, const float* coeffs, int ns_steps, cudaStream_t st) {
+  const Plan& P = h->plan;
+  for (const GroupPlan& g : P.groups) {
+    prof_begin(h, st);
+    cudaError_t e = launch_tf32_split(reinterpret_cast<float*>(h->ws + g.off_x[0]),
+                                      reinterpret_cast<float*>(h->ws + g.off_xlo[0]), (size_t)g.n * g.s * g.ld_x, st);
+    prof_end(h, MUON_KIND_MOMENTUM_NORM, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "3xTF32 split launch");
+    h->last_launches++;
+  }
+  Tc32Params* tp = new (std::nothrow) Tc32Params();
+  if (!tp) return fail(h, MUON_ERR_OOM, "host allocation of the 3xTF32 launch parameters failed");
+  auto f = [&](size_t off) { return reinterpret_cast<float*>(h->ws + off); };
+  for (int k = 0; k < ns_steps; ++k) {
+    const int cur = k & 1;
+    const float* c = coeffs ? coeffs + 3 * k : kDefaultCoeffs;
+    for (int ph = 0; ph < 3; ++ph) {
+      for (const ChunkPlan& ch : P.chunks) {
+        std::memset(tp, 0, sizeof(Tc32Params));
+        for (int gg = ch.g_begin; gg < ch.g_end; ++gg) {
+          const int li = gg - ch.g_begin;
+          const GroupPlan& g = P.groups[gg];
+          Tc32Group& t = tp->g[li];
+          t.s = g.s; t.L = g.L; t.gid_base = g.gid_base;
+          const size_t xs = (size_t)g.s * g.ld_x, ss = (size_t)g.s * g.ld_s;
+          if (ph == kPhaseGram) {
+            tp->a_hi[li] = P.t_xk[0][cur][gg];
+            tp->a_lo[li] = P.t_xk[1][cur][gg];
+            t.out_hi = f(g.off_gram); t.out_lo = f(g.off_gram_lo); t.ld_out = g.ld_s; t.out_stride = ss;
+          } else if (ph == kPhasePoly) {
+            tp->a_hi[li] = P.t_gram[0][gg];
+            tp->a_lo[li] = P.t_gram[1][gg];
+            t.in_hi = f(g.off_gram); t.in_lo = f(g.off_gram_lo); t.ld_in = g.ld_s; t.in_stride = ss;
+            t.out_hi = f(g.off_poly); t.out_lo = f(g.off_poly_lo); t.ld_out = g.ld_s; t.out_stride = ss;
+          } else {
+            tp->a_hi[li] = P.t_poly[0][gg];
+            tp->a_lo[li] = P.t_poly[1][gg];
+            tp->b_hi[li] = P.t_xmn[0][cur][gg];
+            tp->b_lo[li] = P.t_xmn[1][cur][gg];
+            t.in_hi = f(g.off_x[cur]); t.in_lo = f(g.off_xlo[cur]); t.ld_in = g.ld_x; t.in_stride = xs;
+            t.out_hi = f(g.off_x[cur ^ 1]); t.out_lo = f(g.off_xlo[cur ^ 1]); t.ld_out = g.ld_x; t.out_stride = xs;
+          }
+        }
+        tp->tiles = reinterpret_cast<const TcTile*>(h->ws + P.off_tiles) + ch.off_tiles[ph];
+        tp->n_tiles = ch.n_tiles[ph];
+        tp->first_iter = (k == 0) ? 1 : 0;
+        tp->plain_out = (ph == kPhaseUpdate && k == ns_steps - 1) ? 1 : 0;
+        tp->ca = c[0];
+        tp->cb = c[1];
+        tp->cc = c[2];
+        tp->scale = f(P.off_scale);
+        tp->status = h->dev_status;
+        prof_begin(h, st);
+        const cudaError_t e = launch_tc32(ph, *tp, st);
+        prof_end(h, MUON_KIND_GRAM + ph, st);
+        if (e != cudaSuccess) {
+          delete tp;
+          return cuda_fail(h, e, "3xTF32 Newton-Schulz launch");
+        }
+        h->last_launches++;
+      }
+    }
+  }
+  delete tp;
+  return MUON_OK;
+}
+
 // fuse_cm: caller matrices whose weight update is fused into the last Update pass
 // (nullptr: the last pass stores X_K for a separate apply / export pass).
 muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, const std::vector<CallMat>* fuse_cm,
@@ -844,7 +957,8 @@ muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, const s
   const Plan& P = h->plan;
   if (use_persistent(h, P)) return launch_ns_persistent(h, coeffs, ns_steps, fuse_cm, cautious, st);
   float* scale = reinterpret_cast<float*>(h->ws + P.off_scale);
-  if (P.mode == MUON_MODE_FP32_VALIDATE) {
+  if (P.mode == MUON_MODE_FP32_VALIDATE) return launch_ns_tf32x3(h, coeffs, ns_steps, st);
+  if (P.mode == MUON_MODE_FP32_SIMT) {
     for (int k = 0; k < ns_steps; ++k) {
       const int cur = k & 1;
       const float* c = coeffs ? coeffs + 3 * k : kDefaultCoeffs;
@@ -1066,7 +1180,7 @@ muon_status step_impl(muon_handle_t h, const muon_matrix* mats, int n, float lr,
   if (!finite(momentum) || momentum < 0.f || momentum >= 1.f)
     return fail(h, MUON_ERR_INVALID_ARG, "momentum must lie in [0, 1)");
   if (!finite(eps) || eps < 0.f) return fail(h, MUON_ERR_INVALID_ARG, "eps must be finite and >= 0");
-  if (mode != MUON_MODE_BF16 && mode != MUON_MODE_FP32_VALIDATE)
+  if (mode != MUON_MODE_BF16 && mode != MUON_MODE_FP32_VALIDATE && mode != MUON_MODE_FP32_SIMT)
     return fail(h, MUON_ERR_INVALID_ARG, "unknown mode %d", (int)mode);
   muon_status s = check_coeffs(h, coeffs, ns_steps);
   if (s) return s;
@@ -1152,7 +1266,7 @@ muon_status muon_newton_schulz(muon_handle_t h, const void* const* x_in, void* c
   if (!x_in || !o_out || !rows || !cols) return fail(h, MUON_ERR_INVALID_ARG, "NULL array argument");
   if (dtype != MUON_F32 && dtype != MUON_BF16) return fail(h, MUON_ERR_INVALID_ARG, "unknown dtype");
   if (!finite(eps) || eps < 0.f) return fail(h, MUON_ERR_INVALID_ARG, "eps must be finite and >= 0");
-  if (mode != MUON_MODE_BF16 && mode != MUON_MODE_FP32_VALIDATE)
+  if (mode != MUON_MODE_BF16 && mode != MUON_MODE_FP32_VALIDATE && mode != MUON_MODE_FP32_SIMT)
     return fail(h, MUON_ERR_INVALID_ARG, "unknown mode %d", (int)mode);
   muon_status s = check_coeffs(h, coeffs, ns_steps);
   if (s) return s;

@@ -211,7 +211,7 @@ struct __align__(64) TcPersistParams {
   CUtensorMap gram_out[kMaxGroupsPersist];// Gram 32 x 32 blocks: Gram output, Poly epilogue input
   CUtensorMap poly[kMaxGroupsPersist];    // Poly K-major: Update A operand
   CUtensorMap poly_out[kMaxGroupsPersist];// Poly 32 x 32 blocks: Poly output
-  TcGroup g[kMaxGroupsPersist];
+  TcGroup g[kMaxGroupsPersist];    // x_cur / x_next: the X buffers of even / odd steps
   const TcTile* tiles_syrk;        // Gram and Poly tiles (cost-sorted), n_syrk entries
   const TcTile* tiles_upd;         // Update tiles (cost-sorted), n_upd entries
   int n_syrk, n_upd;
@@ -270,7 +270,48 @@ inline int tc_update_tiles(int s, int L, uint16_t group, uint16_t mat, TcTile* o
   return n;
 }
 
-// ----------------------------------------------------------------- fp32 validation path
+// ----------------------------------------------------------------- fp32 validation, tensor cores
+//
+// fp32 storage and 3xTF32 products on tcgen05 (kind::tf32): every fp32 value x of X, the
+// Gram matrix and the polynomial matrix is kept as hi = tf32(x) and lo = tf32(x - hi)
+// (both rounded to nearest; hi + lo holds 22 significant bits of x), and each product
+// accumulates hi*hi + hi*lo + lo*hi in fp32 in tensor memory.  Tile lists, tile shapes and the operand layouts in shared
+// memory are those of the bf16 engine, with 32 fp32 (one 128-byte swizzle row) per
+// k-block.  The last Update stores its value unsplit, for the weight-update / export
+// pass.
+struct Tc32Group {
+  int s, L;              // matrix in wide orientation: s x L
+  int gid_base;          // global index of matrix 0 of the group
+  int ld_in, ld_out;     // leading dimensions (elements) of the epilogue input and output
+  size_t in_stride, out_stride;  // elements between consecutive matrices of the group
+  const float* in_hi;    // epilogue input: Gram (Poly) or X_cur (Update), hi and lo parts
+  const float* in_lo;
+  float* out_hi;         // output: Gram, Poly or X_next, hi and lo parts
+  float* out_lo;
+};
+
+struct __align__(64) Tc32Params {
+  CUtensorMap a_hi[kMaxGroups];  // A operand, K-major, box 32 x 128 (Gram: X; Poly: Gram; Update: Poly)
+  CUtensorMap a_lo[kMaxGroups];
+  CUtensorMap b_hi[kMaxGroups];  // Update B operand: X, MN-major, box 32 x 32
+  CUtensorMap b_lo[kMaxGroups];
+  Tc32Group g[kMaxGroups];
+  const TcTile* tiles;
+  int n_tiles;
+  int first_iter;                // fold the Frobenius scale into this pass
+  int plain_out;                 // last Update: store the value unsplit into out_hi
+  float ca, cb, cc;
+  const float* scale;
+  int* status;
+};
+static_assert(sizeof(Tc32Params) <= 32764, "3xTF32 parameters must fit the kernel parameter space");
+
+// One grouped launch of one phase (k_tc_tf32.cu).
+cudaError_t launch_tc32(int phase, const Tc32Params& p, cudaStream_t st);
+// In place hi = tf32(x), and lo = tf32(x - hi), over n floats (the momentum pass's X0).
+cudaError_t launch_tf32_split(float* hi, float* lo, size_t n, cudaStream_t st);
+
+// ----------------------------------------------------------------- fp32 validation, CUDA cores
 
 struct F32Mat {
   float* x_cur;

@@ -86,7 +86,8 @@ SHAPES = [(300, 130), (130, 301), (256, 256), (513, 257), (64, 1000), (1000, 517
 
 
 @pytest.mark.parametrize("table", [TABLE5, TABLE6], ids=["5rows", "6rows"])
-@pytest.mark.parametrize("mode,dtype,tol", [("fp32", torch.float32, F32_TOL), ("bf16", torch.bfloat16, BF16_TOL)])
+@pytest.mark.parametrize("mode,dtype,tol", [("fp32", torch.float32, F32_TOL), ("fp32_simt", torch.float32, F32_TOL),
+                                            ("bf16", torch.bfloat16, BF16_TOL)])
 def test_newton_schulz_table_rows_differ(mb, handle, mode, dtype, tol, table):
     """Grouped muon_newton_schulz with a table whose rows differ, and with the same rows
     reversed: each matches the oracle run with its own table, and the two differ."""
@@ -103,7 +104,7 @@ def test_newton_schulz_table_rows_differ(mb, handle, mode, dtype, tol, table):
         assert rel(to64(orv), to64(o)) > 0.1, tuple(x.shape)
 
 
-@pytest.mark.parametrize("mode,tol", [("fp32", F32_TOL), ("bf16", BF16_TOL)])
+@pytest.mark.parametrize("mode,tol", [("fp32", F32_TOL), ("fp32_simt", F32_TOL), ("bf16", BF16_TOL)])
 def test_step_table_rows_differ(mb, handle, mode, tol):
     """Two whole steps (momentum, normalisation, Newton-Schulz, update) of the tiny set
     with the 5-row table: momentum bit for bit, weight change against the oracle."""

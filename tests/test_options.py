@@ -167,7 +167,7 @@ def normuon_run(mb, data, states, steps, **kw):
     return [(-w / sc) for w, sc in zip(W, scales)], M
 
 
-@pytest.mark.parametrize("mode,tol", [("bf16", BF16_TOL), ("fp32", 1e-4)])
+@pytest.mark.parametrize("mode,tol", [("bf16", BF16_TOL), ("fp32", 1e-4), ("fp32_simt", 1e-4)])
 def test_normuon_two_steps_vs_oracle(mb, mode, tol):
     if mode == "bf16":
         data = synth.make_matrix_set(1, device="cuda", layers=[0])
