@@ -44,6 +44,12 @@
  *  - With the environment variable MUON_LOG set (and not "0") when a handle is
  *    created, that handle writes its plans (shape groups, tile counts, workspace
  *    bytes) and the detail of every error to stderr.
+ *  - With MUON_DEBUG set (and not "0") when a handle is created, that handle puts a
+ *    256-byte guard band filled with a fixed pattern after every workspace region, and
+ *    at the end of every call (outside stream capture) waits for the call's work and
+ *    checks the bands on the device: a changed band is returned as MUON_ERR_CORRUPT,
+ *    naming the region it follows, and the bands are filled again.  Results are the
+ *    same as without it; calls then synchronize the stream.
  */
 #ifndef MUON_B200_MUON_H
 #define MUON_B200_MUON_H
@@ -69,7 +75,8 @@ typedef enum {
   MUON_ERR_OOM = 3,          /* workspace allocation failed */
   MUON_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed */
   MUON_ERR_TIMEOUT = 5,      /* a bounded device-side wait expired (kernel gave up and returned) */
-  MUON_ERR_TOO_LARGE = 6     /* the matrix does not fit the fixed scratch of muon_newton_schulz_noalloc */
+  MUON_ERR_TOO_LARGE = 6,    /* the matrix does not fit the fixed scratch of muon_newton_schulz_noalloc */
+  MUON_ERR_CORRUPT = 7       /* debug mode: a guard band around a workspace region was overwritten */
 } muon_status;
 
 typedef enum { MUON_F32 = 0, MUON_BF16 = 1 } muon_dtype;
@@ -264,6 +271,12 @@ MUON_API muon_status muon_set_launch_mode(muon_handle_t h, muon_launch_mode mode
  * working.  No device work by itself.  Returns MUON_ERR_INVALID_ARG for a NULL handle
  * or a limit out of range. */
 MUON_API muon_status muon_selftest_stall_persistent(muon_handle_t h, int64_t limit_ns);
+
+/* Diagnostic for the debug mode's guard check: overwrites one byte of the last guard
+ * band of the handle's workspace (synchronously, with cudaMemset), so that the next
+ * call returns MUON_ERR_CORRUPT.  Returns MUON_ERR_INVALID_ARG for a NULL handle, a
+ * handle not in debug mode or one without a workspace yet. */
+MUON_API muon_status muon_selftest_corrupt_guard(muon_handle_t h);
 
 /* Diagnostic for the allocation-failure path: the next time the handle must allocate
  * its workspace (a call with a new list of shapes or mode that needs more than the

@@ -26,6 +26,7 @@ MUON_ERR_OOM = 3
 MUON_ERR_CUDA = 4
 MUON_ERR_TIMEOUT = 5
 MUON_ERR_TOO_LARGE = 6
+MUON_ERR_CORRUPT = 7
 
 MUON_F32 = 0
 MUON_BF16 = 1
@@ -36,6 +37,7 @@ MUON_MODE_FP32_SIMT = 2
 EXPORTED = ("muon_init", "muon_step", "muon_step_ex", "muon_newton_schulz", "muon_newton_schulz_noalloc",
             "muon_sync",
             "muon_selftest_wait_timeout", "muon_selftest_fail_next_alloc", "muon_selftest_stall_persistent",
+            "muon_selftest_corrupt_guard",
             "muon_set_launch_mode",
             "muon_workspace_bytes",
             "muon_last_launch_count", "muon_profile_enable", "muon_profile_read", "muon_destroy",
@@ -99,6 +101,8 @@ def load_library(path: str = LIB_PATH):
     lib.muon_newton_schulz_noalloc.restype = i32
     lib.muon_selftest_wait_timeout.argtypes = [vp, i64, vp]
     lib.muon_selftest_wait_timeout.restype = i32
+    lib.muon_selftest_corrupt_guard.argtypes = [vp]
+    lib.muon_selftest_corrupt_guard.restype = i32
     lib.muon_selftest_stall_persistent.argtypes = [vp, i64]
     lib.muon_selftest_stall_persistent.restype = i32
     lib.muon_set_launch_mode.argtypes = [vp, i32]
@@ -321,6 +325,12 @@ def muon_selftest_stall_persistent(handle, limit_ns: int) -> None:
     handle's next persistent launch gives up after limit_ns and the next muon_sync raises
     MuonError with code MUON_ERR_TIMEOUT."""
     _check(load_library().muon_selftest_stall_persistent(handle, int(limit_ns)), handle)
+
+
+def muon_selftest_corrupt_guard(handle) -> None:
+    """Overwrites one byte of a guard band of a debug-mode handle (MUON_DEBUG=1 when it was
+    created); the next call raises MuonError with code MUON_ERR_CORRUPT."""
+    _check(load_library().muon_selftest_corrupt_guard(handle), handle)
 
 
 def muon_selftest_fail_next_alloc(handle) -> None:

@@ -85,6 +85,10 @@ struct Plan {
   std::vector<CUtensorMap> map_xout[2], map_gram_out, map_poly_out;
   // 3xTF32 mode (fp32): X K-major and MN-major, Gram, Poly; hi and lo parts
   std::vector<CUtensorMap> t_xk[2][2], t_xmn[2][2], t_gram[2], t_poly[2];
+  // debug mode: guard bands after every workspace region (offset, region name), their
+  // offsets on the device, and the check's result words
+  std::vector<std::pair<size_t, const char*>> guards;
+  size_t off_guard_table = 0, off_guard_result = 0;
 };
 
 }  // namespace
@@ -129,6 +133,9 @@ struct muon_handle {
   TcPersistParams* persist = nullptr;  // host staging of the persistent launch's parameters
   // MUON_LOG set (and not "0") at muon_init: plan summaries and errors go to stderr
   bool log = false;
+  // MUON_DEBUG set (and not "0") at muon_init: guard bands around workspace regions,
+  // checked after every call
+  bool debug = false;
 };
 
 namespace {
@@ -243,6 +250,60 @@ muon_status encode_map(muon_handle* h, CUtensorMap* map, void* base, int inner, 
   return MUON_OK;
 }
 
+// ------------------------------------------------------------------ debug mode: guard bands
+
+constexpr size_t kGuardBytes = 256;
+constexpr unsigned char kGuardByte = 0xA5;
+
+// One block per guard band: counts the bytes that no longer hold the pattern, and
+// records the lowest index of a band that changed.
+__global__ void guard_check_kernel(const unsigned char* ws, const uint64_t* offs, int n, unsigned* result) {
+  const int gi = blockIdx.x;
+  if (gi >= n) return;
+  const unsigned char* g = ws + offs[gi];
+  unsigned bad = 0;
+  for (int i = threadIdx.x; i < (int)kGuardBytes; i += blockDim.x) bad += g[i] != kGuardByte ? 1u : 0u;
+  if (bad) {
+    atomicAdd(&result[0], bad);
+    atomicMin(&result[1], (unsigned)gi);
+  }
+}
+
+// Fills every guard band with the pattern.
+cudaError_t arm_guards(muon_handle* h, cudaStream_t st) {
+  for (const auto& g : h->plan.guards) {
+    const cudaError_t e = cudaMemsetAsync(h->ws + g.first, kGuardByte, kGuardBytes, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+// Debug mode, after a call's work: waits for it, checks every guard band and reports an
+// overwritten one as MUON_ERR_CORRUPT (the bands are then filled again).
+muon_status check_guards(muon_handle* h, cudaStream_t st) {
+  const Plan& P = h->plan;
+  if (!h->debug || P.guards.empty()) return MUON_OK;
+  unsigned* res = reinterpret_cast<unsigned*>(h->ws + P.off_guard_result);
+  cudaError_t e = cudaMemsetAsync(res, 0, 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(res + 1, 0xFF, 4, st);
+  if (e == cudaSuccess) {
+    guard_check_kernel<<<(unsigned)P.guards.size(), 128, 0, st>>>(
+        reinterpret_cast<const unsigned char*>(h->ws), reinterpret_cast<const uint64_t*>(h->ws + P.off_guard_table),
+        (int)P.guards.size(), res);
+    e = cudaGetLastError();
+  }
+  unsigned host[2] = {0, 0};
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpy(host, res, sizeof(host), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(h, e, "guard band check");
+  if (host[0] == 0) return MUON_OK;
+  const char* what = host[1] < P.guards.size() ? P.guards[host[1]].second : "?";
+  if ((e = arm_guards(h, st)) == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(h, e, "guard band re-arm");
+  return fail(h, MUON_ERR_CORRUPT, "%u bytes of the guard bands changed; the first one follows the %s", host[0],
+              what);
+}
+
 muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols, int n, muon_mode mode,
                        cudaStream_t st) {
   Plan& P = h->plan;
@@ -309,26 +370,39 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
   // workspace layout
   size_t off = 0;
   const bool tf32x3 = mode == MUON_MODE_FP32_VALIDATE;
+  // Places a region of `bytes` at the next multiple of `align`; in debug mode a guard
+  // band follows its last byte (at the next 16-byte boundary).
+  auto place = [&](size_t bytes, size_t align, const char* what) {
+    off = align_up(off, align);
+    const size_t o = off;
+    off += bytes;
+    if (h->debug) {
+      off = align_up(off, 16);
+      P.guards.push_back({off, what});
+      off += kGuardBytes;
+    }
+    return o;
+  };
   for (auto& g : P.groups) {
     const size_t xbytes = (size_t)g.n * g.s * g.ld_x * esz;
     const size_t sbytes = (size_t)g.n * g.s * g.ld_s * esz;
-    g.off_x[0] = off; off = align_up(off + xbytes, 1024);
-    g.off_x[1] = off; off = align_up(off + xbytes, 1024);
-    g.off_gram = off; off = align_up(off + sbytes, 1024);
-    g.off_poly = off; off = align_up(off + sbytes, 1024);
+    g.off_x[0] = place(xbytes, 1024, "X (even steps)");
+    g.off_x[1] = place(xbytes, 1024, "X (odd steps)");
+    g.off_gram = place(sbytes, 1024, "Gram matrices");
+    g.off_poly = place(sbytes, 1024, "polynomial matrices");
     if (tf32x3) {
-      g.off_xlo[0] = off; off = align_up(off + xbytes, 1024);
-      g.off_xlo[1] = off; off = align_up(off + xbytes, 1024);
-      g.off_gram_lo = off; off = align_up(off + sbytes, 1024);
-      g.off_poly_lo = off; off = align_up(off + sbytes, 1024);
+      g.off_xlo[0] = place(xbytes, 1024, "X lo parts (even steps)");
+      g.off_xlo[1] = place(xbytes, 1024, "X lo parts (odd steps)");
+      g.off_gram_lo = place(sbytes, 1024, "Gram lo parts");
+      g.off_poly_lo = place(sbytes, 1024, "polynomial lo parts");
     }
   }
-  P.off_partials = off; off = align_up(off + (size_t)P.total_units * kWarpsPerUnit * 4, 256);
-  P.off_scale = off; off = align_up(off + (size_t)n * 4, 256);
-  P.off_rowsq = off; off = align_up(off + (size_t)P.total_rows * 4, 256);
-  P.off_rowf = off; off = align_up(off + (size_t)P.total_rows * 4, 256);
+  P.off_partials = place((size_t)P.total_units * kWarpsPerUnit * 4, 1024, "norm partials");
+  P.off_scale = place((size_t)n * 4, 256, "norm scales");
+  P.off_rowsq = place((size_t)P.total_rows * 4, 256, "NorMuon row sums");
+  P.off_rowf = place((size_t)P.total_rows * 4, 256, "NorMuon row factors");
   // persistent launch: work counter + one completed-tile counter per matrix
-  P.off_sched = off; off = align_up(off + (size_t)(1 + n) * 4, 256);
+  P.off_sched = place((size_t)(1 + n) * 4, 256, "persistent-launch counters");
   // tile lists (tensor-core paths)
   if (mode != MUON_MODE_FP32_SIMT) {
     for (int g0 = 0; g0 < (int)P.groups.size(); g0 += kMaxGroups) {
@@ -358,9 +432,13 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
       P.chunks.push_back(c);
     }
   }
-  P.off_tiles = off;
-  off = align_up(off + P.tiles.size() * sizeof(TcTile), 256);
-  P.bytes = off;
+  P.off_tiles = place(P.tiles.size() * sizeof(TcTile), 256, "tile lists");
+  if (h->debug) {
+    P.off_guard_table = align_up(off, 256);
+    P.off_guard_result = align_up(P.off_guard_table + P.guards.size() * 8, 256);
+    off = P.off_guard_result + 256;
+  }
+  P.bytes = align_up(off, 256);
 
   // (re)allocate the workspace
   if (P.bytes > h->ws_bytes) {
@@ -389,6 +467,14 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
     if (e != cudaSuccess) return cuda_fail(h, e, "tile list upload");
     e = cudaStreamSynchronize(st);  // the host vector must outlive the copy
     if (e != cudaSuccess) return cuda_fail(h, e, "tile list upload");
+  }
+  if (h->debug) {
+    std::vector<uint64_t> table(P.guards.size());
+    for (size_t i = 0; i < P.guards.size(); ++i) table[i] = P.guards[i].first;
+    if (!table.empty()) e = cudaMemcpy(h->ws + P.off_guard_table, table.data(), table.size() * 8, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = arm_guards(h, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "guard band set-up");
   }
   if (mode == MUON_MODE_BF16) {
     const size_t ng = P.groups.size();
@@ -1082,6 +1168,10 @@ muon_status finish_call(muon_handle* h, cudaStream_t st) {
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   cudaStreamIsCapturing(st, &cs);
   if (cs != cudaStreamCaptureStatusNone) return MUON_OK;
+  if (h->debug) {
+    const muon_status g = check_guards(h, st);
+    if (g != MUON_OK) return g;
+  }
   cudaError_t e = cudaMemcpyAsync(h->host_status, h->dev_status, sizeof(int), cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaEventRecord(h->status_event, st);
   if (e != cudaSuccess) return cuda_fail(h, e, "status copy");
@@ -1151,6 +1241,8 @@ muon_status muon_init(muon_handle_t* out, int device) {
   h->encode = reinterpret_cast<EncodeTiledFn>(fn);
   const char* lg = getenv("MUON_LOG");
   h->log = lg != nullptr && lg[0] != '\0' && strcmp(lg, "0") != 0;
+  const char* dbg = getenv("MUON_DEBUG");
+  h->debug = dbg != nullptr && dbg[0] != '\0' && strcmp(dbg, "0") != 0;
   if (h->log) fprintf(stderr, "muon: handle on device %d (%s, %d SMs)\n", device, prop.name, h->sm_count);
   *out = h;
   return MUON_OK;
@@ -1333,6 +1425,19 @@ muon_status muon_selftest_stall_persistent(muon_handle_t h, int64_t limit_ns) {
   return MUON_OK;
 }
 
+muon_status muon_selftest_corrupt_guard(muon_handle_t h) {
+  if (!h) return MUON_ERR_INVALID_ARG;
+  h->err.clear();
+  if (!h->debug || !h->plan.valid || h->plan.guards.empty())
+    return fail(h, MUON_ERR_INVALID_ARG, "no guard bands: the handle is not in debug mode or has no workspace yet");
+  DeviceGuard dg(h->device);
+  if (!dg.ok) return fail(h, MUON_ERR_CUDA, "cannot select device %d", h->device);
+  const size_t last = h->plan.guards.size() - 1;
+  const cudaError_t e = cudaMemset(h->ws + h->plan.guards[last].first + 3, 0, 1);
+  if (e != cudaSuccess) return cuda_fail(h, e, "guard band write");
+  return MUON_OK;
+}
+
 muon_status muon_selftest_fail_next_alloc(muon_handle_t h) {
   if (!h) return MUON_ERR_INVALID_ARG;
   h->fail_next_alloc = true;
@@ -1414,6 +1519,7 @@ const char* muon_status_string(muon_status s) {
     case MUON_ERR_CUDA: return "MUON_ERR_CUDA: CUDA call failed";
     case MUON_ERR_TIMEOUT: return "MUON_ERR_TIMEOUT: a device-side wait timed out";
     case MUON_ERR_TOO_LARGE: return "MUON_ERR_TOO_LARGE: matrix exceeds the fixed scratch of the allocation-free entry point";
+    case MUON_ERR_CORRUPT: return "MUON_ERR_CORRUPT: a workspace guard band was overwritten (debug mode)";
     default: return "unknown muon_status";
   }
 }

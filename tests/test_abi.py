@@ -36,10 +36,11 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(6):
-        assert mb.muon_status_string(code).startswith(
-            ["MUON_OK", "MUON_ERR_INVALID_ARG", "MUON_ERR_UNSUPPORTED", "MUON_ERR_OOM", "MUON_ERR_CUDA",
-             "MUON_ERR_TIMEOUT"][code])
+    names = ["MUON_OK", "MUON_ERR_INVALID_ARG", "MUON_ERR_UNSUPPORTED", "MUON_ERR_OOM", "MUON_ERR_CUDA",
+             "MUON_ERR_TIMEOUT", "MUON_ERR_TOO_LARGE", "MUON_ERR_CORRUPT"]
+    for code, name in enumerate(names):
+        assert mb.muon_status_string(code).startswith(name)
+        assert getattr(mb, name) == code
     assert "unknown" in mb.muon_status_string(99)
 
 
@@ -49,6 +50,10 @@ def test_null_handle_is_rejected_before_any_device_call(lib):
     assert lib.muon_newton_schulz(None, None, None, None, None, 0, 1, None, 5, 1e-7, 0, None) \
         == mb.MUON_ERR_INVALID_ARG
     assert lib.muon_sync(None) == mb.MUON_ERR_INVALID_ARG
+    assert lib.muon_set_launch_mode(None, 0) == mb.MUON_ERR_INVALID_ARG
+    assert lib.muon_selftest_fail_next_alloc(None) == mb.MUON_ERR_INVALID_ARG
+    assert lib.muon_selftest_stall_persistent(None, 1000) == mb.MUON_ERR_INVALID_ARG
+    assert lib.muon_selftest_corrupt_guard(None) == mb.MUON_ERR_INVALID_ARG
     assert lib.muon_workspace_bytes(None) == 0
     assert lib.muon_last_error(None) == b""
     out = ctypes.c_void_p()

@@ -181,3 +181,83 @@ def test_log_environment_variable_reports_plans_and_errors():
     env["MUON_LOG"] = "0"
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and "muon:" not in r.stderr
+
+
+# ---------------------------------------------------------------- debug mode: workspace guard bands
+
+def _debug_handle(mb, mode="auto"):
+    import os
+    old = os.environ.get("MUON_DEBUG")
+    os.environ["MUON_DEBUG"] = "1"
+    try:
+        h = mb.muon_init(0)
+    finally:
+        if old is None:
+            del os.environ["MUON_DEBUG"]
+        else:
+            os.environ["MUON_DEBUG"] = old
+    mb.muon_set_launch_mode(h, mode)
+    return h
+
+
+@pytest.mark.parametrize("launch,mode", [("phases", "bf16"), ("persistent", "bf16"), ("auto", "fp32"),
+                                         ("auto", "fp32_simt")])
+def test_debug_guard_bands_stay_intact_and_results_match(mb, launch, mode):
+    """A debug-mode handle (guard bands after every workspace region, checked after every
+    call) gives the same bits as a plain handle, and no band changes: on a depth-8 layer
+    and on ragged shapes, through muon_step and muon_newton_schulz."""
+    import synth
+    data = synth.make_matrix_set(1, layers=[0])
+    G = [g.cuda() for g in data["G"]]
+    ragged = [(300, 130), (130, 301), (7, 1003), (45, 45)]
+    xs = [synth.random_matrix(r, c, seed=50 + i, device="cuda", dtype=torch.bfloat16 if mode == "bf16"
+                              else torch.float32) for i, (r, c) in enumerate(ragged)]
+    outs = {}
+    for debug in (False, True):
+        h = _debug_handle(mb, launch) if debug else mb.muon_init(0)
+        try:
+            if not debug:
+                mb.muon_set_launch_mode(h, launch)
+            W = [w.cuda().clone() for w in data["W"]]
+            M = [m.cuda().clone() for m in data["M"]]
+            for _ in range(2):
+                mb.muon_step(h, W, G, M, lr=0.02, mode=mode)
+            o = [torch.empty_like(x) for x in xs]
+            mb.muon_newton_schulz(h, xs, o, mode=mode)
+            torch.cuda.synchronize()
+            mb.muon_sync(h)
+            outs[debug] = (W, M, o, mb.muon_workspace_bytes(h))
+        finally:
+            mb.muon_destroy(h)
+    for a, b in zip(outs[False][0] + outs[False][1] + outs[False][2], outs[True][0] + outs[True][1] + outs[True][2]):
+        assert torch.equal(a, b)
+    assert outs[True][3] > outs[False][3]  # the bands take room
+
+
+def test_debug_guard_detects_an_overwritten_band(mb):
+    """One byte of a guard band is overwritten on purpose (a memset, on the host's
+    request): the next call reports MUON_ERR_CORRUPT naming the region, re-arms the
+    bands, and the call after it is clean."""
+    h = _debug_handle(mb)
+    try:
+        w = torch.zeros(256, 64, device="cuda")
+        g = torch.randn(256, 64, device="cuda")
+        m = torch.zeros(256, 64, device="cuda")
+        mb.muon_step(h, [w], [g], [m], lr=0.1)
+        mb.muon_selftest_corrupt_guard(h)
+        with pytest.raises(mb.MuonError) as e:
+            mb.muon_step(h, [w], [g], [m], lr=0.1)
+        assert e.value.code == mb.MUON_ERR_CORRUPT
+        assert "guard" in str(e.value) and "follows the tile lists" in str(e.value)
+        mb.muon_step(h, [w], [g], [m], lr=0.1)
+        torch.cuda.synchronize()
+        mb.muon_sync(h)
+    finally:
+        mb.muon_destroy(h)
+    h = mb.muon_init(0)
+    try:
+        with pytest.raises(mb.MuonError) as e:
+            mb.muon_selftest_corrupt_guard(h)
+        assert e.value.code == mb.MUON_ERR_INVALID_ARG
+    finally:
+        mb.muon_destroy(h)
