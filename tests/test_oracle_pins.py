@@ -78,6 +78,22 @@ def pin_spectral_map(ns):
         assert np.allclose(sv_got, sv_want, rtol=1e-11, atol=1e-13)
 
 
+# An invented per-step table whose rows differ (the pages give the triples per step but
+# print none): each row's scalar map stays bounded on (0, 1.3].
+TABLE_ROWS_DIFFER = [QUINTIC, tuple(0.9 * v for v in QUINTIC), CUBIC, (2.0, -1.5, 0.5), (3.0, -3.2, 1.2)]
+
+
+def pin_spectral_map_table(ns):
+    """With row k of a table used in step k, O = U diag(f_K(...f_1(s))) V^T: the steps'
+    scalar maps compose in the table's order (closed form of the iteration)."""
+    for (rows, cols, seed) in [(24, 9, 6), (9, 24, 7), (20, 20, 8)]:
+        x, _ = conditioned(rows, cols, seed, lo=0.02, hi=1.0)
+        u, s, vt = np.linalg.svd(x, full_matrices=False)
+        want = (u * scalar_map(s, TABLE_ROWS_DIFFER)) @ vt
+        got = ns(x, TABLE_ROWS_DIFFER)
+        assert rel(got, want) < 1e-11, (rows, cols, rel(got, want))
+
+
 def pin_polar(ns):
     """Cubic triple iterated to convergence = the SVD polar factor U V^T."""
     for (rows, cols, seed) in [(8, 5, 11), (5, 8, 12), (16, 16, 13), (12, 3, 14)]:
@@ -104,7 +120,7 @@ def pin_transpose(ns):
         assert rel(a, b) < 1e-13, (rows, cols)
 
 
-PINS = [pin_diagonal, pin_spectral_map, pin_polar, pin_transpose]
+PINS = [pin_diagonal, pin_spectral_map, pin_spectral_map_table, pin_polar, pin_transpose]
 
 
 # ---------------------------------------------------------------- the pins on the oracle
@@ -276,7 +292,12 @@ def _mutant(kind):
     def ns(x0, coeffs):
         x = np.array(x0, dtype=np.float64, copy=True)
         tall = x.shape[0] > x.shape[1]
-        for a, b, c in coeffs:
+        rows = list(coeffs)
+        if kind == "reverse_rows":
+            rows = rows[::-1]
+        if kind == "first_row_only":
+            rows = [rows[0]] * len(rows)
+        for a, b, c in rows:
             if kind == "drop_c":
                 c = 0.0
             if kind == "sign_b":
@@ -293,7 +314,7 @@ def _mutant(kind):
     return ns
 
 
-@pytest.mark.parametrize("kind", ["drop_c", "sign_b", "swap_side", "drop_a"])
+@pytest.mark.parametrize("kind", ["drop_c", "sign_b", "swap_side", "drop_a", "reverse_rows", "first_row_only"])
 def test_pins_catch_planted_mistakes(kind):
     bad = _mutant(kind)
     caught = 0
