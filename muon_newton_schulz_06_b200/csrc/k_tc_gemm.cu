@@ -816,25 +816,45 @@ tc_persistent_kernel(const __grid_constant__ TcPersistParams p, const __grid_con
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (uint32_t j = 0; ok; ++j) {
-        int item;
-        if (rank == 0) {
-          const uint32_t slot = j % kSched, par = (j / kSched) & 1u;
-          if (!mbar_wait_cluster(&sched_empty[slot], par ^ 1u, abort_flag)) { ok = false; break; }
-          item = (int)atomicAdd(p.queue, 1u);
-          if (item >= n_items) item = -1;
-          sched_item[slot] = item;
-          st_cluster_u32(peer_addr(smem_u32(&sched_item[slot]), 1), (uint32_t)item);
-          mbar_arrive_local(&sched_full[slot]);
-          remote_arrive(peer_addr(smem_u32(&sched_full[slot]), 1));
-        } else {
-          if (!take_item(j, item, true)) { ok = false; break; }
-        }
-        if (item < 0) break;
-        const PItem it = decode_item(p, item);
+      // Item j of this cluster: the leader takes it from the global counter and publishes
+      // it; the peer reads it from the ring.
+      auto next_item = [&](uint32_t j, int& item) -> bool {
+        if (rank != 0) return take_item(j, item, true);
+        const uint32_t slot = j % kSched, par = (j / kSched) & 1u;
+        if (!mbar_wait_cluster(&sched_empty[slot], par ^ 1u, abort_flag)) return false;
+        item = (int)atomicAdd(p.queue, 1u);
+        if (item >= n_items) item = -1;
+        sched_item[slot] = item;
+        st_cluster_u32(peer_addr(smem_u32(&sched_item[slot]), 1), (uint32_t)item);
+        mbar_arrive_local(&sched_full[slot]);
+        remote_arrive(peer_addr(smem_u32(&sched_full[slot]), 1));
+        return true;
+      };
+      // The next item is taken as soon as the current one's inputs are complete, and its
+      // own inputs are polled while the current one's loads wait for free stages, so its
+      // first loads go out as soon as a stage frees.
+      int cur = -1;
+      bool cur_ready = false;  // cur's inputs already seen complete (acquire done)
+      if (!next_item(0, cur)) ok = false;
+      for (uint32_t j = 0; ok && cur >= 0; ++j) {
+        const PItem it = decode_item(p, cur);
         const TcGroup& g = p.g[it.tile.group];
-        if (!wait_item_deps(p, g, g.gid_base + it.tile.mat, it.k, it.ph, abort_flag)) { ok = false; break; }
+        if (!cur_ready && !wait_item_deps(p, g, g.gid_base + it.tile.mat, it.k, it.ph, abort_flag)) {
+          ok = false;
+          break;
+        }
         fence_async_global();
+        int nxt = -1;
+        if (!next_item(j + 1, nxt)) { ok = false; break; }
+        bool nxt_ready = false;
+        const unsigned* nxt_ctr = nullptr;
+        unsigned nxt_target = 0;
+        if (nxt >= 0) {
+          const PItem itn = decode_item(p, nxt);
+          const TcGroup& gn = p.g[itn.tile.group];
+          nxt_ctr = p.done + gn.gid_base + itn.tile.mat;
+          nxt_target = item_target(p, gn, gn.gid_base + itn.tile.mat, itn.k, itn.ph);
+        }
         const bool syrk = it.ph != kPhaseUpdate;
         const int K = (it.ph == kPhaseGram) ? g.L : g.s;
         const int nk = (K + kBK - 1) / kBK;
@@ -845,7 +865,10 @@ tc_persistent_kernel(const __grid_constant__ TcPersistParams p, const __grid_con
         const int row_a = it.tile.bi * kTile + (int)rank * kHalf;
         const int col_b = it.tile.bj * kTile + (int)rank * kHalf;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_try_wait(&empty[stage], phase ^ 1u)) {
+            if (nxt_ctr != nullptr && !nxt_ready) nxt_ready = ld_acquire_gpu(nxt_ctr) >= nxt_target;
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          }
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], kPairTxBytes);
           const uint32_t a_dst = smem_u32(smem + stage * kStageBytes);
           const uint32_t b_dst = a_dst + kABytes;
@@ -861,6 +884,8 @@ tc_persistent_kernel(const __grid_constant__ TcPersistParams p, const __grid_con
           }
           if (++stage == kPStages) { stage = 0; phase ^= 1u; }
         }
+        cur = nxt;
+        cur_ready = nxt_ready;
       }
       if (!ok || *abort_flag) {
         give_up();

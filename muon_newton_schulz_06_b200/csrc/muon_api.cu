@@ -64,6 +64,9 @@ struct MatPlan {
 struct ChunkPlan {
   int g_begin = 0, g_end = 0;
   size_t off_tiles[3] = {0, 0, 0};
+  // the persistent launch's lists (symmetric products, update): every phase in one
+  // matrix priority, larger L first, so a matrix's next phase follows its previous one
+  size_t off_ptiles[2] = {0, 0};
   int n_tiles[3] = {0, 0, 0};
 };
 
@@ -226,12 +229,22 @@ muon_status check_coeffs(muon_handle* h, const float* coeffs, int ns_steps) {
 
 // ------------------------------------------------------------------ plan
 
+// Per-phase launches: each list longest contraction first (Gram by L, Poly and Update by
+// s), for the balance of one launch's waves.
 void sort_tiles(std::vector<TcTile>& t, const std::vector<GroupPlan>& groups, int phase) {
   auto cost = [&](const TcTile& x) {
     const GroupPlan& g = groups[x.group];
     return (int64_t)(phase == kPhaseGram ? g.L : g.s);
   };
   std::stable_sort(t.begin(), t.end(), [&](const TcTile& a, const TcTile& b) { return cost(a) > cost(b); });
+}
+
+// Persistent launch: the same matrix priority in every phase (larger L first, the
+// matrices with the longest Gram contraction and the most update tiles), so the items of
+// a matrix's next phase come up in the order its previous phase completes.
+void sort_tiles_persistent(std::vector<TcTile>& t, const std::vector<GroupPlan>& groups) {
+  std::stable_sort(t.begin(), t.end(),
+                   [&](const TcTile& a, const TcTile& b) { return groups[a.group].L > groups[b.group].L; });
 }
 
 muon_status encode_map(muon_handle* h, CUtensorMap* map, void* base, int inner, int rows, int n, int ld,
@@ -428,6 +441,12 @@ muon_status build_plan(muon_handle* h, const int64_t* rows, const int64_t* cols,
         c.off_tiles[ph] = P.tiles.size();
         c.n_tiles[ph] = (int)lists[ph].size();
         P.tiles.insert(P.tiles.end(), lists[ph].begin(), lists[ph].end());
+      }
+      std::vector<TcTile> plists[2] = {syrk, upd};
+      for (int q = 0; q < 2; ++q) {
+        sort_tiles_persistent(plists[q], cg);
+        c.off_ptiles[q] = P.tiles.size();
+        P.tiles.insert(P.tiles.end(), plists[q].begin(), plists[q].end());
       }
       P.chunks.push_back(c);
     }
@@ -937,8 +956,8 @@ muon_status launch_ns_persistent(muon_handle* h, const float* coeffs, int ns_ste
     pp.poly_out[li] = P.map_poly_out[gg];
   }
   const TcTile* dev_tiles = reinterpret_cast<const TcTile*>(h->ws + P.off_tiles);
-  pp.tiles_syrk = dev_tiles + ch.off_tiles[kPhaseGram];
-  pp.tiles_upd = dev_tiles + ch.off_tiles[kPhaseUpdate];
+  pp.tiles_syrk = dev_tiles + ch.off_ptiles[0];
+  pp.tiles_upd = dev_tiles + ch.off_ptiles[1];
   pp.n_syrk = ch.n_tiles[kPhaseGram];
   pp.n_upd = ch.n_tiles[kPhaseUpdate];
   pp.ns_steps = ns_steps;

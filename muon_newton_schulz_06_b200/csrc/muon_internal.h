@@ -197,9 +197,9 @@ struct __align__(16) TcApplyTable {
 // epilogue warp of a pair adds 1 to the matrix's counter once its part of a tile is
 // stored, so phase p of step k of a matrix with nS symmetric and nU update tiles may
 // start once the counter reaches kArrivalsPerTile * (k*(2 nS + nU) + [p >= 1] nS +
-// [p >= 2] nS).  The tile lists and their order are those of the per-phase launches,
-// and each tile's products and epilogue arithmetic are the same, so results are
-// bit-identical to launch_tc's.
+// [p >= 2] nS).  The tiles are those of the per-phase launches (listed in one matrix
+// priority for every phase, larger L first), and each tile's products and epilogue
+// arithmetic are the same, so results are bit-identical to launch_tc's.
 constexpr int kMaxNsStepsDev = 16;
 // Shape groups of one persistent launch (ten tensor maps per group travel with it).
 constexpr int kMaxGroupsPersist = 8;

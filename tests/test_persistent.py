@@ -266,3 +266,38 @@ def test_persistent_abort_path_reports_timeout_and_recovers(mb):
         assert torch.equal(a, b)
     lib = mb.load_library()
     assert lib.muon_selftest_stall_persistent(None, 1000) == mb.MUON_ERR_INVALID_ARG
+
+
+def test_persistent_launches_on_two_streams_at_once(mb):
+    """Two handles run persistent steps on two streams at the same time, so the two
+    launches compete for the SMs and neither can count on all its clusters being
+    resident.  Work items are handed out in order, so both finish (no time-out) and
+    each gives the bits of the same steps run alone."""
+    sets = [synth.make_matrix_set(1, layers=[0]), synth.make_matrix_set(2, layers=[0])]
+    alone, together = [], []
+    for data in sets:
+        W = [w.cuda().clone() for w in data["W"]]
+        M = [m.cuda().clone() for m in data["M"]]
+        run_steps(mb, "persistent", W, [g.cuda() for g in data["G"]], M, steps=3, lr=0.02)
+        alone.append((W, M))
+    hs = [handle(mb, "persistent") for _ in sets]
+    streams = [torch.cuda.Stream() for _ in sets]
+    try:
+        state = []
+        for data in sets:
+            state.append(([w.cuda().clone() for w in data["W"]], [g.cuda() for g in data["G"]],
+                          [m.cuda().clone() for m in data["M"]]))
+        torch.cuda.synchronize()
+        for _ in range(3):
+            for h, st, (W, G, M) in zip(hs, streams, state):
+                mb.muon_step(h, W, G, M, lr=0.02, stream=st)
+        torch.cuda.synchronize()
+        for h in hs:
+            mb.muon_sync(h)
+        together = [(W, M) for W, _, M in state]
+    finally:
+        for h in hs:
+            mb.muon_destroy(h)
+    for (wa, ma), (wt, mt) in zip(alone, together):
+        for a, b in zip(wa + ma, wt + mt):
+            assert torch.equal(a, b)
