@@ -13,7 +13,7 @@ value      algorithmic Newton-Schulz TFLOP (one triangle of the symmetric produc
            per step x steps, summed over ranks, / the slowest rank's device time of
            the whole steps (CUDA events on the launch stream).
 e2e        the same metric when every step also copies the gradients in from pinned
-           host memory and the updated weights back out; the step is issued as four
+           host memory and the updated weights back out; the step is issued as eight
            calls over layer runs so the copies overlap compute (--e2e-chunks).
 roofline   the kernel with the largest share of device time, from per-launch CUDA
            events the library records on its stream during the timed steps.
@@ -36,7 +36,7 @@ if ROOT not in sys.path:
 METRIC = "Muon step ms & NS TFLOP/s (fraction of bf16 tensor peak) per model matrix set, 1 B200"
 UNIT = "TFLOP/s"
 LR, MU, EPS, NS_STEPS = 0.02, 0.95, 1e-7, 5
-E2E_CHUNKS = 4  # calls per step in the end-to-end pipeline (transfers overlap within a step)
+E2E_CHUNKS = 8  # calls per step in the end-to-end pipeline (transfers overlap within a step)
 WORKLOAD_TEXT = {
     1: "d8: depth-8 GPT, d_model 512, MLP 2048, 48 bf16 matrices",
     2: "d12: depth-12 GPT, d_model 768, MLP 3072, 72 bf16 matrices",
