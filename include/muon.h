@@ -50,6 +50,9 @@
  *    checks the bands on the device: a changed band is returned as MUON_ERR_CORRUPT,
  *    naming the region it follows, and the bands are filled again.  Results are the
  *    same as without it; calls then synchronize the stream.
+ *  - With MUON_NVTX set (and not "0") when a handle is created, that handle wraps every
+ *    call and every kernel launch in an NVTX range named after the call or the kernel
+ *    kind, for timeline profilers (no effect on results).
  */
 #ifndef MUON_B200_MUON_H
 #define MUON_B200_MUON_H

@@ -20,6 +20,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "muon.h"
 #include "muon_internal.h"
 
@@ -139,6 +141,9 @@ struct muon_handle {
   // MUON_DEBUG set (and not "0") at muon_init: guard bands around workspace regions,
   // checked after every call
   bool debug = false;
+  // MUON_NVTX set (and not "0") at muon_init: an NVTX range around every call and every
+  // kernel launch, for timeline profilers
+  bool nvtx = false;
 };
 
 namespace {
@@ -175,13 +180,23 @@ cudaEvent_t take_event(muon_handle* h) {
 }
 
 // Brackets one launch with events on its stream while profiling is on.
-void prof_begin(muon_handle* h, cudaStream_t st) {
+// Name of a kernel kind in the NVTX ranges (muon_kernel_kind order).
+const char* kind_name(int kind) {
+  static const char* const names[MUON_KIND_COUNT] = {"muon momentum/norm", "muon Gram",   "muon polynomial",
+                                                     "muon update",        "muon apply",  "muon update+apply",
+                                                     "muon persistent Newton-Schulz"};
+  return kind >= 0 && kind < MUON_KIND_COUNT ? names[kind] : "muon";
+}
+
+void prof_begin(muon_handle* h, cudaStream_t st, int kind) {
+  if (h->nvtx) nvtxRangePushA(kind_name(kind));
   if (!h->profiling) return;
   h->ev_open = take_event(h);
   if (h->ev_open) cudaEventRecord(h->ev_open, st);
 }
 
 void prof_end(muon_handle* h, int kind, cudaStream_t st) {
+  if (h->nvtx) nvtxRangePop();
   if (!h->profiling || !h->ev_open) return;
   cudaEvent_t b = take_event(h);
   if (!b) return;
@@ -854,7 +869,7 @@ muon_status launch_elementwise(muon_handle* h, const std::vector<CallMat>& cm, i
     ep->total_units = units;
     const int grid = std::max(1, std::min(units, h->sm_count * 8));
     int launches = pass == kPassOut ? 1 : 2;
-    prof_begin(h, st);
+    prof_begin(h, st, pass == kPassMomentum ? MUON_KIND_MOMENTUM_NORM : MUON_KIND_APPLY);
     cudaError_t err;
     if (pass == kPassMomentum && ep->use_momentum && !f32) {
       err = launch_momentum_bf16(h, *ep, b, &launches, st);
@@ -976,7 +991,7 @@ muon_status launch_ns_persistent(muon_handle* h, const float* coeffs, int ns_ste
   if (fuse_cm) fill_apply_table(h, ch, *fuse_cm, cautious);
   const int n_items = ns_steps * (2 * pp.n_syrk + pp.n_upd);
   const int clusters = std::max(1, std::min(tc_persistent_clusters(), n_items));
-  prof_begin(h, st);
+  prof_begin(h, st, MUON_KIND_NS_PERSISTENT);
   cudaError_t e = cudaMemsetAsync(pp.queue, 0, (size_t)(1 + P.mats.size()) * 4, st);
   if (e == cudaSuccess) e = launch_tc_persistent(pp, fuse_cm ? h->apply_table : nullptr, clusters, st);
   prof_end(h, MUON_KIND_NS_PERSISTENT, st);
@@ -991,7 +1006,7 @@ muon_status launch_ns_persistent(muon_handle* h, const float* coeffs, int ns_ste
 muon_status launch_ns_tf32x3(muon_handle* h, const float* coeffs, int ns_steps, cudaStream_t st) {
   const Plan& P = h->plan;
   for (const GroupPlan& g : P.groups) {
-    prof_begin(h, st);
+    prof_begin(h, st, MUON_KIND_MOMENTUM_NORM);
     cudaError_t e = launch_tf32_split(reinterpret_cast<float*>(h->ws + g.off_x[0]),
                                       reinterpret_cast<float*>(h->ws + g.off_xlo[0]), (size_t)g.n * g.s * g.ld_x, st);
     prof_end(h, MUON_KIND_MOMENTUM_NORM, st);
@@ -1040,7 +1055,7 @@ muon_status launch_ns_tf32x3(muon_handle* h, const float* coeffs, int ns_steps, 
         tp->cc = c[2];
         tp->scale = f(P.off_scale);
         tp->status = h->dev_status;
-        prof_begin(h, st);
+        prof_begin(h, st, MUON_KIND_GRAM + ph);
         const cudaError_t e = launch_tc32(ph, *tp, st);
         prof_end(h, MUON_KIND_GRAM + ph, st);
         if (e != cudaSuccess) {
@@ -1076,13 +1091,13 @@ muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, const s
         f.gram = reinterpret_cast<float*>(h->ws + g.off_gram + (size_t)m.idx * g.s * g.ld_s * 4);
         f.poly = reinterpret_cast<float*>(h->ws + g.off_poly + (size_t)m.idx * g.s * g.ld_s * 4);
         f.s = g.s; f.L = g.L; f.ld_x = g.ld_x; f.ld_s = g.ld_s; f.gid = g.gid_base + m.idx;
-        prof_begin(h, st);
+        prof_begin(h, st, MUON_KIND_GRAM);
         cudaError_t e = launch_f32_gram(f, k == 0, scale, st);
         prof_end(h, MUON_KIND_GRAM, st);
-        prof_begin(h, st);
+        prof_begin(h, st, MUON_KIND_POLY);
         if (e == cudaSuccess) e = launch_f32_poly(f, c[1], c[2], st);
         prof_end(h, MUON_KIND_POLY, st);
-        prof_begin(h, st);
+        prof_begin(h, st, MUON_KIND_UPDATE);
         if (e == cudaSuccess) e = launch_f32_update(f, k == 0, scale, c[0], st);
         prof_end(h, MUON_KIND_UPDATE, st);
         if (e != cudaSuccess) return cuda_fail(h, e, "fp32 Newton-Schulz launch");
@@ -1133,11 +1148,11 @@ muon_status launch_ns(muon_handle* h, const float* coeffs, int ns_steps, const s
         cudaError_t e = cudaSuccess;
         if (fuse_cm && ph == kPhaseUpdate && k == ns_steps - 1) {
           fill_apply_table(h, ch, *fuse_cm, cautious);
-          prof_begin(h, st);
+          prof_begin(h, st, MUON_KIND_UPDATE_APPLY);
           e = launch_tc_update_apply(*tp, *h->apply_table, clusters, st);
           prof_end(h, MUON_KIND_UPDATE_APPLY, st);
         } else {
-          prof_begin(h, st);
+          prof_begin(h, st, MUON_KIND_GRAM + ph);
           e = launch_tc(ph, *tp, clusters, st);
           prof_end(h, MUON_KIND_GRAM + ph, st);
         }
@@ -1198,8 +1213,19 @@ muon_status finish_call(muon_handle* h, cudaStream_t st) {
   return MUON_OK;
 }
 
+muon_status run_impl(muon_handle* h, const std::vector<CallMat>& cm, const int64_t* rows, const int64_t* cols,
+                     bool step, const CallOpts& o, cudaStream_t st);
+
 muon_status run(muon_handle* h, const std::vector<CallMat>& cm, const int64_t* rows, const int64_t* cols,
                 bool step, const CallOpts& o, cudaStream_t st) {
+  if (h->nvtx) nvtxRangePushA(step ? "muon_step" : "muon_newton_schulz");
+  const muon_status s = run_impl(h, cm, rows, cols, step, o, st);
+  if (h->nvtx) nvtxRangePop();
+  return s;
+}
+
+muon_status run_impl(muon_handle* h, const std::vector<CallMat>& cm, const int64_t* rows, const int64_t* cols,
+                     bool step, const CallOpts& o, cudaStream_t st) {
   const float* coeffs = o.coeffs;
   const int ns_steps = o.ns_steps;
   const muon_mode mode = o.mode;
@@ -1262,6 +1288,8 @@ muon_status muon_init(muon_handle_t* out, int device) {
   h->log = lg != nullptr && lg[0] != '\0' && strcmp(lg, "0") != 0;
   const char* dbg = getenv("MUON_DEBUG");
   h->debug = dbg != nullptr && dbg[0] != '\0' && strcmp(dbg, "0") != 0;
+  const char* nv = getenv("MUON_NVTX");
+  h->nvtx = nv != nullptr && nv[0] != '\0' && strcmp(nv, "0") != 0;
   if (h->log) fprintf(stderr, "muon: handle on device %d (%s, %d SMs)\n", device, prop.name, h->sm_count);
   *out = h;
   return MUON_OK;

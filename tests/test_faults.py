@@ -261,3 +261,37 @@ def test_debug_guard_detects_an_overwritten_band(mb):
         assert e.value.code == mb.MUON_ERR_INVALID_ARG
     finally:
         mb.muon_destroy(h)
+
+
+def test_nvtx_ranges_leave_results_unchanged(mb):
+    """MUON_NVTX=1 at handle creation wraps every call and launch in an NVTX range (seen
+    by a timeline profiler when one is attached); the results keep their bits."""
+    import os
+    import synth
+    data = synth.make_matrix_set(1, layers=[0])
+    G = [g.cuda() for g in data["G"]]
+    outs = []
+    for nvtx in ("0", "1"):
+        old = os.environ.get("MUON_NVTX")
+        os.environ["MUON_NVTX"] = nvtx
+        try:
+            h = mb.muon_init(0)
+        finally:
+            if old is None:
+                del os.environ["MUON_NVTX"]
+            else:
+                os.environ["MUON_NVTX"] = old
+        try:
+            W = [w.cuda().clone() for w in data["W"]]
+            M = [m.cuda().clone() for m in data["M"]]
+            mb.muon_profile_enable(h, True)
+            mb.muon_step(h, W, G, M, lr=0.02)
+            torch.cuda.synchronize()
+            mb.muon_sync(h)
+            prof = mb.muon_profile_read(h)
+            outs.append((W, M, sum(n for _, n in prof.values())))
+        finally:
+            mb.muon_destroy(h)
+    for a, b in zip(outs[0][0] + outs[0][1], outs[1][0] + outs[1][1]):
+        assert torch.equal(a, b)
+    assert outs[0][2] == outs[1][2] > 0
