@@ -74,7 +74,7 @@ typedef struct muon_handle* muon_handle_t;
 typedef enum {
   MUON_OK = 0,
   MUON_ERR_INVALID_ARG = 1,  /* null / misaligned / overlapping pointers, bad sizes or values */
-  MUON_ERR_UNSUPPORTED = 2,  /* a combination this build does not implement (e.g. no sm_100 device) */
+  MUON_ERR_UNSUPPORTED = 2,  /* a combination the library does not implement (e.g. no sm_100 device) */
   MUON_ERR_OOM = 3,          /* workspace allocation failed */
   MUON_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed */
   MUON_ERR_TIMEOUT = 5,      /* a bounded device-side wait expired (kernel gave up and returned) */
