@@ -126,3 +126,51 @@ def test_llama3p8b_full_set_sampled(mb):
                            np.multiply(lrs, O[i].cpu().numpy().astype(np.float32), dtype=np.float32),
                            dtype=np.float32)
         assert torch.equal(Wb[i].cpu(), torch.from_numpy(want).to(torch.bfloat16)), names[i]
+
+
+def test_gpt_full_set_fp32_validation_mode(mb):
+    """Depth-8 set (48 matrices, bf16 gradients) in one call in the fp32 validation mode
+    (3xTF32 on the tensor cores): O within 1e-4 of the oracle, momentum bit-exact."""
+    data = synth.make_matrix_set(1, device="cuda")
+    specs = data["specs"]
+    scales = [math.sqrt(max(1.0, s.rows / s.cols)) for s in specs]
+    W = [torch.zeros(s.rows, s.cols, device="cuda") for s in specs]
+    M = [m.clone() for m in data["M"]]
+    h = mb.muon_init(0)
+    try:
+        mb.muon_step(h, W, data["G"], M, lr=1.0, momentum=0.95, nesterov=True, mode="fp32")
+        torch.cuda.synchronize()
+        mb.muon_sync(h)
+    finally:
+        mb.muon_destroy(h)
+    for i, spec in enumerate(specs):
+        m_ref, _ = oracle.nesterov_momentum_f32(data["G"][i].float().cpu().numpy(), data["M"][i].cpu().numpy(),
+                                                0.95, True)
+        assert np.array_equal(M[i].cpu().numpy(), m_ref), spec
+        o = (-W[i] / scales[i]).double().cpu().numpy()
+        err = rel(o, oracle_o(data["G"][i], data["M"][i]))
+        assert err < 1e-4, (spec, err)
+
+
+@pytest.mark.parametrize("config,layers", [(2, None), (3, [0])])
+def test_launch_forms_agree_on_whole_sets(mb, config, layers):
+    """The whole depth-12 set and a heavy-tailed depth-24 layer: one launch per phase and
+    one persistent launch give the same weights and momentum, bit for bit, over two
+    steps."""
+    data = synth.make_matrix_set(config, device="cuda", layers=layers)
+    out = {}
+    for form in ("phases", "persistent"):
+        W = [w.clone() for w in data["W"]]
+        M = [m.clone() for m in data["M"]]
+        h = mb.muon_init(0)
+        try:
+            mb.muon_set_launch_mode(h, form)
+            for _ in range(2):
+                mb.muon_step(h, W, data["G"], M, lr=0.02, momentum=0.95, nesterov=True)
+            torch.cuda.synchronize()
+            mb.muon_sync(h)
+        finally:
+            mb.muon_destroy(h)
+        out[form] = (W, M)
+    for a, b in zip(out["phases"][0] + out["phases"][1], out["persistent"][0] + out["persistent"][1]):
+        assert torch.equal(a, b)
