@@ -88,7 +88,10 @@ typedef enum {
   MUON_MODE_BF16 = 0,           /* Newton-Schulz on tcgen05 tensor cores, bf16 operands, fp32 accumulate */
   MUON_MODE_FP32_VALIDATE = 1,  /* fp32 storage; products on tcgen05 tensor cores as 3xTF32: each fp32
                                    value is split into hi = tf32(x) and lo = tf32(x - hi) and a
-                                   product accumulates hi*hi + hi*lo + lo*hi in fp32 (validation) */
+                                   product accumulates hi*hi and hi*lo + lo*hi in fp32 (validation).
+                                   The tensor cores' accumulation error grows with the contraction
+                                   length, so a call with a matrix side above 8192 runs on CUDA
+                                   cores as in MUON_MODE_FP32_SIMT */
   MUON_MODE_FP32_SIMT = 2       /* fp32 storage and fp32 FMA on CUDA cores (validation, slowest) */
 } muon_mode;
 

@@ -22,7 +22,13 @@
 //               swizzle; the MN-major X of Update the 128-byte swizzle with a 32-byte
 //               base, the tensor cores' layout for MN-major 32-bit operands
 //   warp 1      TMEM owner; in the leader CTA the MMA issuer: three MMAs per 8-deep
-//               k-step (hi*hi, hi*lo, lo*hi) into the same accumulator
+//               k-step, hi*hi into one 256-column accumulator and hi*lo, lo*hi into a
+//               second one (the epilogue adds the two, rounding to nearest).  The
+//               tensor cores' fp32 accumulation does not round to nearest and its error
+//               grows with the number of accumulations into the large sum; keeping the
+//               cross terms (2^-11 of it) apart leaves one accumulation per k-step in
+//               the large sum instead of three.  Both accumulators serve one tile, so
+//               the epilogue of a tile does not overlap the next tile's products
 //   warps 2..5  epilogue of this CTA's 128 x 256 half: tcgen05.ld 32 lanes x 32
 //               columns, the phase's arithmetic in fp32, then the hi and lo parts (and,
 //               for Gram / Poly, their mirror below the diagonal) straight to global
@@ -256,7 +262,6 @@ __global__ void __launch_bounds__(kThreads32, 1) tc32_kernel(const __grid_consta
       constexpr uint32_t idesc = make_idesc_tf32(!kSyrk);
       int stage = 0;
       uint32_t phase = 0;
-      int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = cluster; t < p.n_tiles && ok; t += n_clusters) {
@@ -264,9 +269,9 @@ __global__ void __launch_bounds__(kThreads32, 1) tc32_kernel(const __grid_consta
         const Tc32Group& g = p.g[tile.group];
         const int K = (PHASE == kPhaseGram) ? g.L : g.s;
         const int nk = (K + kBK32 - 1) / kBK32;
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&tempty[0], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kTile);
+        const uint32_t d_big = tmem_base, d_small = tmem_base + (uint32_t)kTile;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
@@ -277,16 +282,17 @@ __global__ void __launch_bounds__(kThreads32, 1) tc32_kernel(const __grid_consta
             const uint64_t ah = sdesc(a_hi + k * 32, 16, 1024), al = sdesc(a_lo + k * 32, 16, 1024);
             const uint64_t bh = kSyrk ? sdesc(b_hi + k * 32, 16, 1024) : sdesc_mn32(b_hi + k * 1024, 32 * kBK32 * 4, 512);
             const uint64_t bl = kSyrk ? sdesc(b_lo + k * 32, 16, 1024) : sdesc_mn32(b_lo + k * 1024, 32 * kBK32 * 4, 512);
-            umma_pair_tf32(d_tmem, ah, bh, idesc, (kb > 0 || k > 0) ? 1u : 0u);
-            umma_pair_tf32(d_tmem, ah, bl, idesc, 1u);
-            umma_pair_tf32(d_tmem, al, bh, idesc, 1u);
+            const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+            umma_pair_tf32(d_big, ah, bh, idesc, accum);
+            umma_pair_tf32(d_small, ah, bl, idesc, accum);
+            umma_pair_tf32(d_small, al, bh, idesc, 1u);
           }
           umma_commit_both(&empty[stage]);
           if (++stage == kStages32) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit_both(&tfull[acc]);
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        umma_commit_both(&tfull[0]);
+        acc_phase ^= 1u;
       }
       if (!ok) give_up();
       umma_commit_local(drain);
@@ -296,20 +302,19 @@ __global__ void __launch_bounds__(kThreads32, 1) tc32_kernel(const __grid_consta
     // ------------------------------------------------------------------ epilogue (both CTAs)
     const int quad = warp & 3;
     const uint32_t leader_tempty0 = peer_addr(smem_u32(&tempty[0]), 0);
-    int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
     for (int t = cluster; t < p.n_tiles && ok; t += n_clusters) {
       const TcTile tile = p.tiles[t];
       const Tc32Group& g = p.g[tile.group];
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&tfull[0], acc_phase, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const int s = g.s;
       const int lim = kSyrk ? g.s : g.L;
       const int row0 = tile.bi * kTile + (int)rank * kHalf + 32 * quad;
       const int row = row0 + lane;
       const float sc = p.first_iter ? p.scale[g.gid_base + tile.mat] : 1.f;
-      const uint32_t tbase = tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(acc * kTile);
+      const uint32_t tbase = tmem_base + ((uint32_t)(32 * quad) << 16);
       const float* in_hi = (PHASE == kPhaseGram) ? nullptr : g.in_hi + tile.mat * g.in_stride + (size_t)row * g.ld_in;
       const float* in_lo = (PHASE == kPhaseGram) ? nullptr : g.in_lo + tile.mat * g.in_stride + (size_t)row * g.ld_in;
       float* out_hi = g.out_hi + tile.mat * g.out_stride;
@@ -323,8 +328,11 @@ __global__ void __launch_bounds__(kThreads32, 1) tc32_kernel(const __grid_consta
         while (c_lo < c_hi && tile.bj * kTile + 32 * c_lo + 31 < row0) ++c_lo;
       for (int c = c_lo; c < c_hi; ++c) {
         const int col0 = tile.bj * kTile + 32 * c;
-        float v[32];
-        tmem_ld32(tbase + (uint32_t)(32 * c), v);
+        float v[32], vs[32];
+        tmem_ld32(tbase + (uint32_t)(32 * c), v);                      // hi*hi
+        tmem_ld32(tbase + (uint32_t)kTile + (uint32_t)(32 * c), vs);  // hi*lo + lo*hi
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __fadd_rn(v[j], vs[j]);
         if (PHASE == kPhaseGram) {
           const float alpha = sc * sc;
 #pragma unroll
@@ -373,8 +381,8 @@ __global__ void __launch_bounds__(kThreads32, 1) tc32_kernel(const __grid_consta
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) remote_arrive(leader_tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (lane == 0) remote_arrive(leader_tempty0);
+      acc_phase ^= 1u;
     }
     if (!ok && lane == 0) give_up();
   }

@@ -36,6 +36,19 @@ constexpr int kMaxMatrices = 65535;
 // MUON_LAUNCH_AUTO takes the persistent launch below this algorithmic work of one
 // Newton-Schulz step over all of a call's matrices.
 constexpr double kPersistentMaxFlops = 1e12;
+// MUON_MODE_FP32_VALIDATE runs 3xTF32 on the tensor cores only while every contraction is
+// at most this long: the tensor cores' fp32 accumulation error grows with the number of
+// accumulations (measured on one B200: ~4e-5 relative error of O at 8192, ~9e-5 at
+// 16384, ~1.9e-4 at 32768, against 2-7e-6 on CUDA cores); longer ones run on CUDA cores.
+constexpr int64_t kTf32MaxContraction = 8192;
+
+// The fp32 validation form a call runs in: 3xTF32 unless a matrix is too long for it.
+muon_mode fp32_form(muon_mode mode, const int64_t* rows, const int64_t* cols, int n) {
+  if (mode != MUON_MODE_FP32_VALIDATE) return mode;
+  for (int i = 0; i < n; ++i)
+    if (std::max(rows[i], cols[i]) > kTf32MaxContraction) return MUON_MODE_FP32_SIMT;
+  return mode;
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -1359,6 +1372,7 @@ muon_status step_impl(muon_handle_t h, const muon_matrix* mats, int n, float lr,
                     (float)((double)lr * scale), (float)((double)lr * (double)weight_decay), ns_ptr};
   }
   if ((s = check_overlaps(h, ranges))) return s;
+  mode = fp32_form(mode, rows.data(), cols.data(), n);
   CallOpts o;
   o.mu = momentum;
   o.nesterov = nesterov ? 1 : 0;
@@ -1436,7 +1450,7 @@ muon_status muon_newton_schulz(muon_handle_t h, const void* const* x_in, void* c
   o.coeffs = coeffs;
   o.ns_steps = ns_steps;
   o.eps = eps;
-  o.mode = mode;
+  o.mode = fp32_form(mode, rows, cols, n);
   return run(h, cm, rows, cols, false, o, static_cast<cudaStream_t>(cuda_stream));
 }
 

@@ -407,3 +407,83 @@ def test_fp32_modes_agree_and_bound_the_error(mb, handle):
         assert rel(to64(a), want) < F32_TOL, (tuple(x.shape), rel(to64(a), want))
         assert rel(to64(b), want) < F32_TOL, (tuple(x.shape), rel(to64(b), want))
         assert rel(to64(a), to64(b)) < 5e-5, (tuple(x.shape), rel(to64(a), to64(b)))
+
+
+# ------------------------------------------------------------- extremes
+
+@pytest.mark.parametrize("mode,dtype,tol", [("bf16", torch.bfloat16, BF16_TOL), ("fp32", torch.float32, F32_TOL)])
+def test_extreme_aspect_ratios(mb, handle, mode, dtype, tol):
+    """One row or one column of 16384, and 2 x 8000 / 8000 x 3 (s = 1..3, contractions of
+    up to 256 k-blocks), in one grouped call."""
+    shapes = [(1, 16384), (16384, 1), (2, 8000), (8000, 3)]
+    xs = [synth.random_matrix(r, c, seed=600 + i, device="cuda", dtype=dtype) for i, (r, c) in enumerate(shapes)]
+    outs = ns_gpu(mb, handle, xs, mode)
+    for x, o in zip(xs, outs):
+        err = rel(to64(o), ns_oracle(x, [oracle.QUINTIC] * 5))
+        assert err < tol, (tuple(x.shape), err)
+
+
+@pytest.mark.parametrize("mode,dtype,tol", [("bf16", torch.bfloat16, BF16_TOL), ("fp32", torch.float32, F32_TOL),
+                                            ("fp32_simt", torch.float32, F32_TOL)])
+def test_sixteen_steps(mb, handle, mode, dtype, tol):
+    """The most steps a call takes (16), quintic rows then cubic rows, per-phase launches
+    and both fp32 modes."""
+    table = [oracle.QUINTIC] * 8 + [oracle.CUBIC] * 8
+    shapes = [(300, 130), (256, 256), (130, 700)]
+    xs = [synth.random_matrix(r, c, seed=700 + i, device="cuda", dtype=dtype) for i, (r, c) in enumerate(shapes)]
+    h = mb.muon_init(0)
+    try:
+        mb.muon_set_launch_mode(h, "phases")
+        outs = [torch.empty_like(x) for x in xs]
+        mb.muon_newton_schulz(h, xs, outs, coeffs=table, ns_steps=16, mode=mode)
+        torch.cuda.synchronize()
+        mb.muon_sync(h)
+    finally:
+        mb.muon_destroy(h)
+    for x, o in zip(xs, outs):
+        err = rel(to64(o), ns_oracle(x, table))
+        assert err < tol, (tuple(x.shape), err)
+
+
+@pytest.mark.parametrize("mode", ["bf16", "fp32"])
+def test_nan_gradient_stays_in_its_matrix(mb, mode):
+    """A NaN in one gradient makes that matrix's update NaN (nothing checks for it on the
+    hot path) and leaves the other matrices of the same grouped call, and the next call,
+    exactly as without it."""
+    shapes = [(256, 128), (256, 128), (128, 300)]
+    G = [synth.random_matrix(r, c, seed=800 + i, device="cuda") for i, (r, c) in enumerate(shapes)]
+    Gn = [g.clone() for g in G]
+    Gn[0][3, 5] = float("nan")
+    res = []
+    for grads in (G, Gn, G):
+        W = [torch.zeros(r, c, device="cuda") for r, c in shapes]
+        M = [torch.zeros(r, c, device="cuda") for r, c in shapes]
+        h = mb.muon_init(0)
+        try:
+            mb.muon_step(h, W, grads, M, lr=0.1, mode=mode)
+            torch.cuda.synchronize()
+            mb.muon_sync(h)
+        finally:
+            mb.muon_destroy(h)
+        res.append(W)
+    assert torch.isnan(res[1][0]).all()
+    for i in (1, 2):
+        assert torch.equal(res[0][i], res[1][i])
+    for a, b in zip(res[0], res[2]):
+        assert torch.equal(a, b)
+
+
+def test_fp32_validation_mode_uses_cuda_cores_for_long_contractions(mb, handle):
+    """The 3xTF32 form's accumulation error grows with the contraction length, so the fp32
+    validation mode runs a call whose longest side exceeds 8192 on CUDA cores: the bits of
+    MUON_MODE_FP32_SIMT there, the tensor-core form at 8192; both within 1e-4."""
+    x_long = synth.random_matrix(64, 9000, seed=901, device="cuda")
+    x_edge = synth.random_matrix(64, 8192, seed=902, device="cuda")
+    (a,) = ns_gpu(mb, handle, [x_long], "fp32")
+    (b,) = ns_gpu(mb, handle, [x_long], "fp32_simt")
+    assert torch.equal(a, b)
+    (c,) = ns_gpu(mb, handle, [x_edge], "fp32")
+    (d,) = ns_gpu(mb, handle, [x_edge], "fp32_simt")
+    assert not torch.equal(c, d)  # different arithmetic: the tensor-core form ran
+    for x, o in ((x_long, a), (x_edge, c), (x_edge, d)):
+        assert rel(to64(o), ns_oracle(x, [oracle.QUINTIC] * 5)) < F32_TOL
