@@ -24,7 +24,9 @@
  * Conventions for every entry point
  *  - All matrix pointers are DEVICE pointers on the handle's device, row-major and
  *    contiguous (element (i, j) at i*cols + j), 16-byte aligned.  They stay owned
- *    by the caller.  No two matrices' pointers may overlap.
+ *    by the caller.  No two matrices' pointers may overlap.  A pointer that is not
+ *    device memory of the handle's device (host memory, another GPU's memory) is
+ *    an argument error (checked when a call's pointers differ from the last call's).
  *  - Work is enqueued on `cuda_stream` (a cudaStream_t; NULL = legacy default
  *    stream) and the call returns without waiting for it.
  *  - Argument errors are detected on the host and returned before anything is

@@ -157,6 +157,11 @@ struct muon_handle {
   // MUON_NVTX set (and not "0") at muon_init: an NVTX range around every call and every
   // kernel launch, for timeline profilers
   bool nvtx = false;
+  // the pointer lists of the last two calls that were found to be device memory of
+  // `device` (a call with one of them is not checked again; loops often alternate
+  // between two sets of buffers)
+  std::vector<const void*> checked_ptrs[2];
+  int checked_next = 0;
 };
 
 namespace {
@@ -243,6 +248,26 @@ muon_status check_overlaps(muon_handle* h, std::vector<Range>& rs) {
   for (size_t i = 1; i < rs.size(); ++i)
     if (rs[i].lo < rs[i - 1].hi)
       return fail(h, MUON_ERR_INVALID_ARG, "buffers of matrices %d and %d overlap", rs[i - 1].mat, rs[i].mat);
+  return MUON_OK;
+}
+
+// Every pointer must be device memory (plain or managed) of the handle's device: host
+// memory, or another GPU's, would be read and written by the kernels.  The last two lists
+// that passed are remembered, so a loop over the same buffers pays one comparison each.
+muon_status check_device_pointers(muon_handle* h, const std::vector<const void*>& ptrs) {
+  if (ptrs == h->checked_ptrs[0] || ptrs == h->checked_ptrs[1]) return MUON_OK;
+  for (size_t i = 0; i < ptrs.size(); ++i) {
+    if (i > 0 && ptrs[i] == ptrs[i - 1]) continue;
+    cudaPointerAttributes a;
+    const cudaError_t e = cudaPointerGetAttributes(&a, ptrs[i]);
+    if (e != cudaSuccess) cudaGetLastError();
+    if (e != cudaSuccess || (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) ||
+        a.device != h->device)
+      return fail(h, MUON_ERR_INVALID_ARG, "pointer %zu of the call (%p) is not device memory of device %d", i,
+                  ptrs[i], h->device);
+  }
+  h->checked_ptrs[h->checked_next] = ptrs;
+  h->checked_next ^= 1;
   return MUON_OK;
 }
 
@@ -1372,6 +1397,19 @@ muon_status step_impl(muon_handle_t h, const muon_matrix* mats, int n, float lr,
                     (float)((double)lr * scale), (float)((double)lr * (double)weight_decay), ns_ptr};
   }
   if ((s = check_overlaps(h, ranges))) return s;
+  {
+    std::vector<const void*> ptrs;
+    ptrs.reserve((size_t)n * (normuon ? 4 : 3));
+    for (int i = 0; i < n; ++i) {
+      ptrs.push_back(mats[i].param);
+      ptrs.push_back(mats[i].grad);
+      ptrs.push_back(mats[i].momentum);
+      if (normuon) ptrs.push_back(nstate[i]);
+    }
+    DeviceGuard dg(h->device);
+    if (!dg.ok) return fail(h, MUON_ERR_CUDA, "cannot select device %d", h->device);
+    if ((s = check_device_pointers(h, ptrs))) return s;
+  }
   mode = fp32_form(mode, rows.data(), cols.data(), n);
   CallOpts o;
   o.mu = momentum;
@@ -1445,6 +1483,17 @@ muon_status muon_newton_schulz(muon_handle_t h, const void* const* x_in, void* c
     for (const Range& r : ranges)
       if (lo < r.hi && r.lo < hi)
         return fail(h, MUON_ERR_INVALID_ARG, "output of matrix %d overlaps input of matrix %d", r.mat, i);
+  }
+  {
+    std::vector<const void*> ptrs;
+    ptrs.reserve(2 * (size_t)n);
+    for (int i = 0; i < n; ++i) {
+      ptrs.push_back(x_in[i]);
+      ptrs.push_back(o_out[i]);
+    }
+    DeviceGuard dg(h->device);
+    if (!dg.ok) return fail(h, MUON_ERR_CUDA, "cannot select device %d", h->device);
+    if ((s = check_device_pointers(h, ptrs))) return s;
   }
   CallOpts o;
   o.coeffs = coeffs;

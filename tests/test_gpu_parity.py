@@ -487,3 +487,38 @@ def test_fp32_validation_mode_uses_cuda_cores_for_long_contractions(mb, handle):
     assert not torch.equal(c, d)  # different arithmetic: the tensor-core form ran
     for x, o in ((x_long, a), (x_edge, c), (x_edge, d)):
         assert rel(to64(o), ns_oracle(x, [oracle.QUINTIC] * 5)) < F32_TOL
+
+
+def test_host_memory_is_rejected_by_the_c_abi(mb):
+    """Through the C ABI directly (the binding already refuses CPU tensors): a gradient in
+    pinned or pageable host memory, or an output in host memory, is an argument error
+    returned before anything is enqueued, and the handle keeps working."""
+    import ctypes
+    lib = mb.load_library()
+    h = mb.muon_init(0)
+    try:
+        w = torch.zeros(64, 32, device="cuda")
+        g = torch.randn(64, 32, device="cuda")
+        m = torch.zeros(64, 32, device="cuda")
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        for host in (torch.randn(64, 32).pin_memory(), torch.randn(64, 32)):
+            arr = (mb.muon_matrix * 1)()
+            arr[0] = mb.muon_matrix(w.data_ptr(), host.data_ptr(), m.data_ptr(), 64, 32, mb.MUON_F32, mb.MUON_F32)
+            code = lib.muon_step(h, arr, 1, 0.1, 0.95, 1, None, 5, ctypes.c_float(1e-7), 0, stream)
+            assert code == mb.MUON_ERR_INVALID_ARG
+            assert b"not device memory" in lib.muon_last_error(h)
+        out_host = torch.empty(64, 32).pin_memory()
+        xin = (ctypes.c_void_p * 1)(g.data_ptr())
+        xout = (ctypes.c_void_p * 1)(out_host.data_ptr())
+        rows = (ctypes.c_int64 * 1)(64)
+        cols = (ctypes.c_int64 * 1)(32)
+        assert lib.muon_newton_schulz(h, xin, xout, rows, cols, 1, mb.MUON_F32, None, 5, ctypes.c_float(1e-7), 0,
+                                      stream) == mb.MUON_ERR_INVALID_ARG
+        torch.cuda.synchronize()
+        assert torch.count_nonzero(m) == 0 and torch.count_nonzero(w) == 0
+        mb.muon_step(h, [w], [g], [m], lr=0.1)
+        torch.cuda.synchronize()
+        mb.muon_sync(h)
+        assert torch.equal(m, g)
+    finally:
+        mb.muon_destroy(h)
