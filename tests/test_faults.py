@@ -295,3 +295,80 @@ def test_nvtx_ranges_leave_results_unchanged(mb):
     for a, b in zip(outs[0][0] + outs[0][1], outs[1][0] + outs[1][1]):
         assert torch.equal(a, b)
     assert outs[0][2] == outs[1][2] > 0
+
+
+# ---------------------------------------------------------------- concurrency between handles
+
+_THREADS_SCRIPT = """
+import hashlib, sys, threading, torch
+import muon_newton_schulz_06_b200 as mb, synth
+mode = sys.argv[1]
+sets = [synth.make_matrix_set(1, layers=[0], device="cuda"), synth.make_matrix_set(2, layers=[0], device="cuda")]
+out = [None, None]
+def run(data, i):
+    stream = torch.cuda.Stream()
+    h = mb.muon_init(0)
+    try:
+        mb.muon_set_launch_mode(h, mode)
+        W = [w.clone() for w in data["W"]]
+        M = [m.clone() for m in data["M"]]
+        for _ in range(3):
+            mb.muon_step(h, W, data["G"], M, lr=0.02, stream=stream)
+        stream.synchronize()
+        mb.muon_sync(h)
+        d = hashlib.sha256()
+        for t in W + M:
+            d.update(t.cpu().contiguous().view(torch.uint8).numpy().tobytes())
+        out[i] = d.hexdigest()
+    finally:
+        mb.muon_destroy(h)
+threads = [threading.Thread(target=run, args=(data, i)) for i, data in enumerate(sets)]
+for t in threads: t.start()
+for t in threads: t.join(timeout=300)
+print(out[0], out[1])
+"""
+
+
+@pytest.mark.parametrize("mode", ["phases", "persistent"])
+def test_two_handles_on_two_threads(mb, mode):
+    """Distinct handles may be used from distinct host threads (each on its own stream).
+    In a fresh process, two threads make their first calls at the same time (the
+    per-device set-up runs once, under a lock) and run three steps each; their results
+    have the bits of the same steps run one after the other."""
+    import hashlib
+    import os
+    import subprocess
+    import sys
+    import synth
+    digests = []
+    for cfg in (1, 2):
+        data = synth.make_matrix_set(cfg, layers=[0], device="cuda")
+        h = mb.muon_init(0)
+        try:
+            mb.muon_set_launch_mode(h, mode)
+            W = [w.clone() for w in data["W"]]
+            M = [m.clone() for m in data["M"]]
+            for _ in range(3):
+                mb.muon_step(h, W, data["G"], M, lr=0.02)
+            torch.cuda.synchronize()
+            mb.muon_sync(h)
+        finally:
+            mb.muon_destroy(h)
+        d = hashlib.sha256()
+        for t in W + M:
+            d.update(t.cpu().contiguous().view(torch.uint8).numpy().tobytes())
+        digests.append(d.hexdigest())
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _THREADS_SCRIPT, mode], capture_output=True, text=True, timeout=600,
+                       env=dict(os.environ, PYTHONPATH=root), cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.split() == digests
+
+
+def test_init_rejects_a_device_out_of_range(mb):
+    lib = mb.load_library()
+    import ctypes
+    out = ctypes.c_void_p()
+    assert lib.muon_init(ctypes.byref(out), torch.cuda.device_count() + 3) == mb.MUON_ERR_INVALID_ARG
+    assert lib.muon_init(ctypes.byref(out), -1) == mb.MUON_ERR_INVALID_ARG
+    assert out.value is None
